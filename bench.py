@@ -1,0 +1,467 @@
+#!/usr/bin/env python
+"""Benchmark of the NF4 + double-quant frozen linear layer with LoRA on B200.
+
+Headline (one JSON line on rank 0): forward + backward TFLOP/s of one
+LLaMA-65B-shaped decoder layer's seven projections (hidden 8192, FFN 22016),
+16 x 512 = 8192 tokens, LoRA rank 64, alpha 16, weights NF4 + double-quant.
+A step is, for each projection: the fused forward (dequant-GEMM + LoRA) and the
+backward (dX through the fused dequant-GEMM, dA, dB).  The weights are
+quantized once, before timing, as a model load does; the encode, standalone
+dequant and decode-shaped GEMV are measured beside it under "secondary".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 (torchrun, one rank per GPU) every rank runs an independent replica
+of the same per-GPU workload (weak scaling, no data-path collective); the
+process group is used only for the barrier and the max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "fused NF4+LoRA linear fwd+bwd TFLOP/s and dequant/GEMV GB/s vs B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except OSError:
+        return FALLBACK_PEAKS, "fallback"
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self._t:
+            self._t.join(timeout=5)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------- distributed
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    return rank, local, world, pg
+
+
+def barrier(pg, device=None):
+    if pg is not None:
+        if device is not None:
+            pg.barrier(device_ids=[device.index])
+        else:
+            pg.barrier()
+
+
+def max_over_ranks(pg, value: float, device=None) -> float:
+    if pg is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device if device is not None else "cpu")
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------- our arm
+def layer_flops(wl) -> tuple:
+    total, fused = 0, 0
+    for p in wl.projections:
+        f = workloads.linear_flops(p.n, p.k, wl.m, wl.r)
+        total += f["total"]
+        # FLOPs executed inside the fused dequant-GEMM launches: dense + LoRA up-projection
+        fused += (2 * wl.m * p.n * p.k + 2 * wl.m * wl.r * p.n) + (2 * wl.m * p.n * p.k + 2 * wl.m * wl.r * p.k)
+    return total, fused
+
+
+def prepare_layer(qb, torch, wl, device):
+    """Generate, upload and quantize the layer (untimed: a model load)."""
+    projs = []
+    for i, p in enumerate(wl.projections):
+        w = workloads.weight((p.n, p.k), proj=i)
+        qt = qb.qlora_quantize_nf4_dq(w.to(device))
+        del w
+        X = workloads.activations(wl.m, p.k, i)
+        dY = workloads.grad_output(wl.m, p.n, i)
+        st = dict(p=p, qt=qt, X_host=X.pin_memory(), dY_host=dY.pin_memory(),
+                  X=X.to(device), dY=dY.to(device),
+                  A=workloads.lora_a(wl.r, p.k, i).to(device), B=workloads.lora_b(p.n, wl.r, i).to(device))
+        fw, bw = qb.qlora_linear_workspace_size(p.n, p.k, wl.m, wl.r)
+        st["ws_f"] = torch.empty(fw, dtype=torch.uint8, device=device)
+        st["ws_b"] = torch.empty(bw, dtype=torch.uint8, device=device)
+        st["Y"] = torch.empty(wl.m, p.n, dtype=torch.bfloat16, device=device)
+        st["XA"] = torch.empty(wl.m, wl.r, dtype=torch.float32, device=device)
+        st["dX"] = torch.empty(wl.m, p.k, dtype=torch.bfloat16, device=device)
+        st["dA"] = torch.empty(wl.r, p.k, dtype=torch.float32, device=device)
+        st["dB"] = torch.empty(p.n, wl.r, dtype=torch.float32, device=device)
+        st["dA_host"] = torch.empty(wl.r, p.k, dtype=torch.float32).pin_memory()
+        st["dB_host"] = torch.empty(p.n, wl.r, dtype=torch.float32).pin_memory()
+        projs.append(st)
+    torch.cuda.synchronize()
+    return projs
+
+
+def run_step(qb, wl, projs, events=None):
+    s = wl.s
+    for st in projs:
+        if events is not None:
+            e0, e1 = events.pop()
+            qb.qlora_time_next_gemm(e0, e1)
+        qb.qlora_linear_fwd(st["qt"], st["X"], st["A"], st["B"], s, save_xa=True, Y=st["Y"], XA=st["XA"],
+                            workspace=st["ws_f"])
+        if events is not None:
+            e0, e1 = events.pop()
+            qb.qlora_time_next_gemm(e0, e1)
+        qb.qlora_linear_bwd(st["qt"], st["X"], st["dY"], st["A"], st["B"], s, XA=st["XA"], dX=st["dX"],
+                            dA=st["dA"], dB=st["dB"], workspace=st["ws_b"])
+
+
+def run_step_e2e(qb, wl, projs):
+    """Same step through the public API with inputs copied from pinned host memory
+    and the LoRA gradients read back."""
+    s = wl.s
+    for st in projs:
+        st["X"].copy_(st["X_host"], non_blocking=True)
+        st["dY"].copy_(st["dY_host"], non_blocking=True)
+        qb.qlora_linear_fwd(st["qt"], st["X"], st["A"], st["B"], s, save_xa=True, Y=st["Y"], XA=st["XA"],
+                            workspace=st["ws_f"])
+        qb.qlora_linear_bwd(st["qt"], st["X"], st["dY"], st["A"], st["B"], s, XA=st["XA"], dX=st["dX"],
+                            dA=st["dA"], dB=st["dB"], workspace=st["ws_b"])
+        st["dA_host"].copy_(st["dA"], non_blocking=True)
+        st["dB_host"].copy_(st["dB"], non_blocking=True)
+
+
+def secondary(qb, torch, device, peaks):
+    """Encode / dequant (4096^2 with outliers) and decode GEMV (65B FFN) bandwidths."""
+    out = {}
+    hbm = peaks["hbm_gbs"]
+    # codec: rotate 4 weight sets (4 x 42 MB > L2)
+    sets = [workloads.weight((4096, 4096), proj=j, outliers=True).to(device) for j in range(4)]
+    qts = [qb.qlora_quantize_nf4_dq(w) for w in sets]
+    ws = torch.empty(qb.qlora_nf4_sizes(4096, 4096)["workspace"], dtype=torch.uint8, device=device)
+    outs = [torch.empty(4096, 4096, dtype=torch.bfloat16, device=device) for _ in range(4)]
+    sz = qb.qlora_nf4_sizes(4096, 4096)
+    codec_bytes = 4096 * 4096 * 2 + sz["codes"] + sz["absmax_q"] + sz["absmax_c2"] + 4
+    for name, fn in (("encode_4096x4096", lambda j: qb.qlora_quantize_nf4_dq(sets[j], out=qts[j], workspace=ws)),
+                     ("dequant_4096x4096", lambda j: qb.qlora_dequantize(qts[j], out=outs[j]))):
+        for j in range(8):
+            fn(j % 4)
+        torch.cuda.synchronize()
+        iters = 40
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for j in range(iters):
+            fn(j % 4)
+        e1.record()
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) / 1e3 / iters
+        gbs = codec_bytes / t / 1e9
+        out[name] = {"us": round(t * 1e6, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
+                     "bytes": codec_bytes}
+    stored_bytes = sz["codes"] + sz["absmax_q"] + sz["absmax_c2"] + 4
+    out["bits_per_param"] = round(8 * stored_bytes / (4096 * 4096), 6)
+    del sets, qts, outs
+    # GEMV: 22016x8192 and 8192x22016, 2 weight sets each (> L2), M in {1, 4, 16}
+    for (n, k) in ((22016, 8192), (8192, 22016)):
+        wsets = []
+        for j in range(2):
+            w = workloads.weight((n, k), proj=20 + j).to(device)
+            wsets.append(qb.qlora_quantize_nf4_dq(w))
+            del w
+        A = workloads.lora_a(64, k, 30).to(device)
+        B = workloads.lora_b(n, 64, 30).to(device)
+        szg = qb.qlora_nf4_sizes(n, k)
+        wbytes = szg["codes"] + szg["absmax_q"] + szg["absmax_c2"] + 4 + (A.numel() + B.numel()) * 2
+        for m in (1, 4, 16):
+            X = workloads.activations(m, k, 31).to(device)
+            Y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+            wsz = torch.empty(qb.qlora_linear_workspace_size(n, k, m, 64)[0], dtype=torch.uint8, device=device)
+            call = lambda j: qb.qlora_linear_fwd(wsets[j % 2], X, A, B, 0.25, save_xa=False, Y=Y, workspace=wsz)
+            for j in range(6):
+                call(j)
+            torch.cuda.synchronize()
+            # one CUDA graph of 20 back-to-back calls removes host launch gaps
+            g = torch.cuda.CUDAGraph()
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s):
+                with torch.cuda.graph(g, stream=s):
+                    for j in range(20):
+                        call(j)
+            torch.cuda.synchronize()
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(5):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            t = e0.elapsed_time(e1) / 1e3 / 100
+            byts = wbytes + m * k * 2 + m * n * 2
+            gbs = byts / t / 1e9
+            out[f"gemv_{n}x{k}_m{m}"] = {"us": round(t * 1e6, 2), "GB/s": round(gbs, 1),
+                                         "frac_hbm": round(gbs / hbm, 4), "bytes": byts}
+            del g
+        del wsets
+    return out
+
+
+def cpu_oracle_sample(wl, m_sample: int, projs_idx=None) -> dict:
+    """The oracle (as it stands) on a bounded sample of the same workload: all
+    weights dequantized by the C oracle, then fwd + bwd of m_sample tokens."""
+    import oracle
+    t_quant = time.time()
+    qts = []
+    for i, p in enumerate(wl.projections):
+        if projs_idx is not None and i not in projs_idx:
+            continue
+        w = workloads.weight((p.n, p.k), proj=i)
+        qts.append((i, p, oracle.quantize(workloads.bf16_bits(w))))
+        del w
+    t_quant = time.time() - t_quant
+    t0 = time.time()
+    flops = 0
+    for i, p, qt in qts:
+        Wd = oracle.dequant_tensor(qt)
+        X = workloads.activations(wl.m, p.k, i)[:m_sample].float().numpy()
+        dY = workloads.grad_output(wl.m, p.n, i)[:m_sample].float().numpy()
+        A = workloads.lora_a(wl.r, p.k, i).float().numpy()
+        B = workloads.lora_b(p.n, wl.r, i).float().numpy()
+        oracle.linear_fwd(Wd, X, A, B, wl.s)
+        oracle.linear_bwd(Wd, X, dY, A, B, wl.s)
+        flops += workloads.linear_flops(p.n, p.k, m_sample, wl.r)["total"]
+    t = time.time() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max([x.get("num_threads", 1) for x in threadpool_info()] + [1])
+    except Exception:
+        blas = os.cpu_count()
+    cores = max(blas, int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1)))
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "seconds": round(t, 2), "setup_quantize_seconds": round(t_quant, 2),
+            "sample": f"{m_sample} of {wl.m} tokens of each of {len(qts)} projections of {wl.name}: "
+                      f"C-oracle dequant of the full weights + float64 numpy fwd+bwd"}
+
+
+def bench_ours(args):
+    import torch
+    import bit_nf4_quantized_encode_b200 as qb
+    rank, local, world, pg = dist_setup(args.gpus)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    peaks, peak_kind = load_peaks()
+    wl = workloads.LLAMA65B
+    flops_step, flops_fused_step = layer_flops(wl)
+    projs = prepare_layer(qb, torch, wl, device)
+
+    for _ in range(args.warmup):
+        run_step(qb, wl, projs)
+    torch.cuda.synchronize()
+    assert qb.qlora_read_device_errors() == 0, "device wait timed out during warm-up"
+
+    # timed region: K steps, fused-GEMM launches bracketed by events for the roofline
+    K = args.steps
+    gemm_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(2 * len(projs) * K)]
+    for a, b in gemm_events:          # torch creates the CUDA event on first record
+        a.record()
+        b.record()
+    ev_stack = list(reversed(gemm_events))
+    clocks = ClockSampler(device.index)
+    barrier(pg, device)
+    torch.cuda.synchronize()
+    clocks.start()
+    launches0 = qb.qlora_kernel_launches()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K):
+        run_step(qb, wl, projs, events=ev_stack)
+    e1.record()
+    torch.cuda.synchronize()
+    launches = qb.qlora_kernel_launches() - launches0
+    barrier(pg, device)
+    clk = clocks.stop()
+    t_local = e0.elapsed_time(e1) / 1e3
+    t = max_over_ranks(pg, t_local, device)
+    gemm_ms = [a.elapsed_time(b) for a, b in gemm_events]
+
+    # end to end: host inputs -> device -> fwd+bwd -> gradients back to host
+    Ke = max(2, min(K, 5))
+    run_step_e2e(qb, wl, projs)
+    torch.cuda.synchronize()
+    barrier(pg, device)
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record()
+    for _ in range(Ke):
+        run_step_e2e(qb, wl, projs)
+    x1.record()
+    torch.cuda.synchronize()
+    te = max_over_ranks(pg, x0.elapsed_time(x1) / 1e3, device)
+    h2d = sum(st["X"].numel() * 2 + st["dY"].numel() * 2 for st in projs)
+    d2h = sum(st["dA"].numel() * 4 + st["dB"].numel() * 4 for st in projs)
+    assert qb.qlora_read_device_errors() == 0
+    if pg is not None:                 # every rank takes the same collective steps
+        barrier(pg, device)
+        pg.destroy_process_group()
+    if rank != 0:
+        return
+
+    value = world * K * flops_step / t / 1e12
+    peak_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    fused_avg_s = sum(gemm_ms) / len(gemm_ms) / 1e3
+    fused_flops_launch = flops_fused_step / (2 * len(projs))
+    achieved = fused_flops_launch / fused_avg_s / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(t / K * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded PCG64 normals, bf16), NF4+DQ weights quantized on device before timing",
+        "config": {"workload": wl.name, "projections": [f"{p.name} {p.n}x{p.k}" for p in wl.projections],
+                   "tokens": wl.m, "lora_rank": wl.r, "lora_alpha": wl.alpha, "nf4_blocksize": 64,
+                   "dq_blocksize": 256, "l2": "inputs larger than L2 (3.9 GB of activations per step)",
+                   "parallelism": f"replicas x{world} (no collective)",
+                   "flops_per_step": flops_step},
+        "e2e": {"value": round(world * Ke * flops_step / te / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke},
+        "gpu_launches": launches,
+        "roofline": {"bound": "tensor", "kernel": "k_fused (dequant-GEMM fwd and bwd-dX)",
+                     "achieved": round(achieved, 1), "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak_t, 4), "peak_kind": f"{peak_kind} sustained bf16",
+                     "traffic": None, "avg_launch_ms": round(fused_avg_s * 1e3, 4),
+                     "share_of_step": round(sum(gemm_ms) / 1e3 / t_local, 4)},
+        "clocks": clk,
+    }
+    if not args.skip_secondary:
+        line["secondary"] = secondary(qb, torch, device, peaks)
+    if not args.skip_cpu:
+        line["cpu_baseline"] = cpu_oracle_sample(wl, m_sample=args.cpu_tokens)
+    print(json.dumps(line), flush=True)
+
+
+def bench_reference(args):
+    """The oracle as the reference arm: each step a bounded sample of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = workloads.LLAMA65B
+    for _ in range(args.warmup):
+        cpu_oracle_sample(wl, m_sample=args.ref_tokens, projs_idx={0})
+    vals, secs = [], 0.0
+    last = None
+    for _ in range(args.steps):
+        last = cpu_oracle_sample(wl, m_sample=args.ref_tokens, projs_idx={0})
+        vals.append(last["value"])
+        secs += last["seconds"]
+    value = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(secs / args.steps * 1e3, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "tokens": wl.m, "lora_rank": wl.r},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": last["cores"],
+                             "kind": "oracle", "sample": last["sample"]},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--skip-secondary", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=64, help="token sample of the CPU-oracle baseline")
+    ap.add_argument("--ref-tokens", type=int, default=16, help="token sample per reference-arm step")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        bench_reference(args)
+    else:
+        bench_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,31 @@
+// codec.h -- kernel-side parameter blocks and launchers of the NF4 codec.
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace qlora {
+
+// Bucketed decision table of the encoder, passed by value (kernel parameter).
+// Buckets 33..63 are padding (never reached for finite inputs).
+constexpr int kBuckets = 64;
+struct EncodeTables {
+  float bucket_thr[kBuckets];
+  uint8_t bucket_base[kBuckets];
+};
+
+// The 16 NF4 levels, passed by value.
+struct CodebookParam {
+  float level[16];
+};
+
+cudaError_t launch_encode(const uint16_t* w, int64_t numel, const EncodeTables& tab, uint8_t* codes,
+                          float* c1buf, double* partials, int grid, cudaStream_t stream);
+cudaError_t launch_double_quant(const float* c1buf, int64_t nblocks, const double* partials,
+                                int npartials, uint8_t* q, float* c2, float* mean, int grid,
+                                cudaStream_t stream);
+cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* qabs, const float* c2,
+                           const float* mean, int64_t numel, const CodebookParam& cb, uint16_t* out,
+                           int grid, cudaStream_t stream);
+
+}  // namespace qlora

@@ -1,0 +1,79 @@
+// gemm.h -- launch interfaces of the tcgen05 GEMM kernels.
+//
+//  * fused dequant-GEMM: D[mdim x tokens] = deq(W)-tile (MMA M = 128, built in
+//    shared memory by dequant warps from packed NF4 codes) x activation-tile^T
+//    (MMA N = token tile, loaded by TMA), persistent over (m-tile, token-tile,
+//    k-split) work units, TMEM accumulators double-buffered.  Forward: the
+//    A tile is deq(W) rows (K-major); backward dX: the A tile is deq(W)^T
+//    (MN-major).  The rank-r LoRA up-projection is appended as extra k-steps
+//    whose A operand is the LoRA weight and whose B operand is the (scaled)
+//    rank-r activation.
+//  * skinny GEMM: D[mdim x 64] = A x B^T over a long contraction, both operands
+//    by TMA (K- or MN-major), split-K with fp32 atomic accumulation; used for
+//    the rank-r LoRA contractions X A^T, dY B, dY^T (XA), G^T X.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "codec.h"
+
+namespace qlora {
+
+enum class FusedDir : int { kFwd = 0, kBwd = 1 };
+
+struct FusedArgs {
+  const uint8_t* codes;      // packed NF4 codes of W [nw, kw]
+  const uint8_t* qabs;       // E4M3 block constants
+  const float* c2;           // per-group second-level absmax
+  const float* mean;         // per-tensor mean of the block constants
+  int64_t nw, kw;            // W shape (out, in)
+  int64_t m;                 // token rows
+  const uint16_t* lora_w;    // fwd: LoRA B [nw, r]; bwd: LoRA A [r, kw] (bf16)
+  int r;                     // LoRA rank (multiple of 8)
+  int lora_steps;            // ceil(r / 64) extra k-steps (0 disables the LoRA term)
+  uint16_t* out;             // bf16 output [m, ldo] (split == 1)
+  float* out_acc;            // fp32 accumulation [m, ldo] (split > 1)
+  int64_t ldo;               // fwd nw, bwd kw
+  int64_t mdim;              // MMA-M extent: fwd nw, bwd kw
+  int ksteps;                // main k-steps: contraction / 64 (rounded up)
+  int m_tiles, t_tiles, splits;
+  CodebookParam cb;
+  uint32_t* err;             // device error flag
+};
+
+struct SkinnyArgs {
+  int64_t mdim, ndim;        // D extent (ndim <= 64 per n-tile)
+  int ksteps;                // contraction / 64 (rounded up)
+  int m_tiles, n_tiles, splits;
+  float* acc;                // fp32 [mdim, ld_acc], accumulated with atomics
+  int64_t ld_acc;
+  uint32_t* err;
+};
+
+// Token tile of the fused kernel: 256 for prefill-shaped calls, 16 for
+// decode-shaped calls (M <= 16).
+cudaError_t launch_fused(FusedDir dir, int token_tile, const FusedArgs& args, const CUtensorMap& act,
+                         const CUtensorMap& lora_act, int num_sms, cudaStream_t stream);
+cudaError_t launch_skinny(bool a_mn_major, bool b_mn_major, const SkinnyArgs& args,
+                          const CUtensorMap& a_map, const CUtensorMap& b_map, int num_sms,
+                          cudaStream_t stream);
+
+// out[i * ld_out + j] = T(scale * in[i * ld_in + j]) for j < cols_in, 0 for
+// cols_in <= j < cols_out (i < rows); T is bf16 or fp32.  With `transpose`
+// the element goes to out[j * ld_out + i] instead (cols_out == cols_in).
+cudaError_t launch_convert_bf16(const float* in, int64_t rows, int64_t cols_in, int64_t ld_in,
+                                int64_t cols_out, float scale, uint16_t* out, int64_t ld_out,
+                                cudaStream_t stream);
+cudaError_t launch_convert_f32(const float* in, int64_t rows, int64_t cols, int64_t ld_in, float scale,
+                               bool transpose, float* out, int64_t ld_out, cudaStream_t stream);
+
+// LoRA gradients for few tokens (M <= 16), fp32 throughout on CUDA cores:
+//   dA[j, k] = s * sum_m G[m, j] X[m, k];   dB[n, j] = s * sum_m dY[m, n] XA[m, j]
+cudaError_t launch_small_grads(const float* G, int64_t ld_g, const float* XA, int64_t ld_xa,
+                               const uint16_t* X, const uint16_t* dY, int64_t M, int64_t rows,
+                               int64_t cols, int r, float s, float* dA, float* dB,
+                               cudaStream_t stream);
+
+}  // namespace qlora

@@ -1,0 +1,128 @@
+// nf4_tables.cpp -- the CUDA library's own NF4 codebook and encode tables.
+//
+// Codebook (QLoRA, arXiv:2305.14314, as summarised by automatone "QLoRA paper
+// explained", paragraph "4-bit NormalFloat (NF4)": levels at the quantiles of
+// a standard normal; creativeworksofknowledge "QLoRA: Fine-Tune 70B on One
+// GPU", section "1. NF4": Gaussian-proportional levels, denser near zero).
+// Construction: 8 positive levels at Phi^-1(1/2 + (delta - 1/2) j / 8),
+// j = 1..8, 7 negative levels at -Phi^-1(1/2 + (delta - 1/2) j / 7), j = 1..7,
+// and an exact zero, all divided by Phi^-1(delta), with
+// delta = 1 - (1/30 + 1/32) / 2; evaluated in double and rounded once to float.
+//
+// The inverse normal CDF here is Newton's method on Phi(x) = erfc(-x/sqrt 2)/2
+// with the normal density as derivative -- computed independently of any other
+// implementation, so that comparing tables across implementations is a check.
+#include "nf4_tables.h"
+
+#include <cmath>
+#include <cstring>
+#include <limits>
+#include <mutex>
+
+namespace qlora {
+namespace {
+
+double inv_normal_cdf(double p) {
+  // Newton from 0; Phi is convex for x > 0 and concave for x < 0, so iterates
+  // approach the root monotonically after the first step.
+  double x = 0.0;
+  const double inv_sqrt2pi = 0.39894228040143267794;
+  for (int it = 0; it < 100; ++it) {
+    const double f = 0.5 * std::erfc(-x / std::sqrt(2.0)) - p;
+    const double d = inv_sqrt2pi * std::exp(-0.5 * x * x);
+    const double step = f / d;
+    x -= step;
+    if (std::fabs(step) <= 1e-17 * std::fmax(1.0, std::fabs(x))) break;
+  }
+  return x;
+}
+
+// Smallest float strictly greater than the exact midpoint of a and b.
+float above_midpoint(float a, float b) {
+  const double mid = 0.5 * (static_cast<double>(a) + static_cast<double>(b));  // exact
+  float f = static_cast<float>(mid);
+  if (static_cast<double>(f) <= mid) f = std::nextafter(f, std::numeric_limits<float>::infinity());
+  return f;
+}
+
+// The bucket the encode kernel assigns to n: RN(16 n + 16), computed with one
+// fused multiply-add against 2^23 so that the integer lands in the low bits.
+int bucket_of(float n) {
+  const float v = std::fmaf(n, 16.0f, 16.0f + 8388608.0f);
+  uint32_t u;
+  std::memcpy(&u, &v, 4);
+  return static_cast<int>(u & 63u);
+}
+
+uint32_t ordered_key(float f) {  // monotone map of floats in [-1, 1] to integers
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+float from_key(uint32_t k) {
+  uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+Nf4Tables build() {
+  Nf4Tables t{};
+  const double delta = 1.0 - 0.5 * (1.0 / 30.0 + 1.0 / 32.0);
+  const double top = inv_normal_cdf(delta);
+  for (int j = 1; j <= 7; ++j)
+    t.level[7 - j] = static_cast<float>(-inv_normal_cdf(0.5 + (delta - 0.5) * j / 7.0) / top);
+  t.level[7] = 0.0f;
+  for (int j = 1; j <= 8; ++j)
+    t.level[7 + j] = static_cast<float>(inv_normal_cdf(0.5 + (delta - 0.5) * j / 8.0) / top);
+
+  // Nearest level with ties to the lower index <=> count of thresholds <= n,
+  // where threshold i is the first float past the midpoint of levels i, i+1.
+  for (int i = 0; i < 15; ++i) t.threshold[i] = above_midpoint(t.level[i], t.level[i + 1]);
+
+  // For each bucket find the float interval [lo, hi] of n in [-1, 1] that the
+  // kernel's bucket formula maps to it (monotone, so bisect on float order).
+  t.ok = true;
+  const uint32_t kmin = ordered_key(-1.0f), kmax = ordered_key(1.0f);
+  for (int u = 0; u < kNumBuckets; ++u) {
+    uint32_t lo = kmin, hi = kmax;  // first key with bucket >= u
+    while (lo < hi) {
+      uint32_t mid = lo + (hi - lo) / 2;
+      if (bucket_of(from_key(mid)) >= u) hi = mid; else lo = mid + 1;
+    }
+    const uint32_t first = lo;
+    lo = kmin; hi = kmax;           // first key with bucket >= u + 1
+    if (bucket_of(from_key(kmax)) <= u) {
+      lo = kmax + 1;
+    } else {
+      while (lo < hi) {
+        uint32_t mid = lo + (hi - lo) / 2;
+        if (bucket_of(from_key(mid)) >= u + 1) hi = mid; else lo = mid + 1;
+      }
+    }
+    const uint32_t last = lo - 1;
+    if (first > last) { t.bucket_base[u] = 15; t.bucket_thr[u] = INFINITY; continue; }
+    const float nlo = from_key(first), nhi = from_key(last);
+    int base = 0, inside = 0;
+    float thr = INFINITY;
+    for (int i = 0; i < 15; ++i) {
+      if (t.threshold[i] <= nlo) ++base;
+      else if (t.threshold[i] <= nhi) { ++inside; thr = t.threshold[i]; }
+    }
+    if (inside > 1) t.ok = false;
+    t.bucket_base[u] = static_cast<uint8_t>(base);
+    t.bucket_thr[u] = thr;
+  }
+  return t;
+}
+
+}  // namespace
+
+const Nf4Tables& nf4_tables() {
+  static Nf4Tables tables;
+  static std::once_flag once;
+  std::call_once(once, [] { tables = build(); });
+  return tables;
+}
+
+}  // namespace qlora

@@ -1,0 +1,23 @@
+// nf4_tables.h -- host-side tables of the CUDA library: the NF4 codebook, the
+// decision thresholds between neighbouring levels, and the bucketed lookup
+// table the encode kernel uses to pick a code with one comparison.
+#pragma once
+#include <cstdint>
+
+namespace qlora {
+
+// Buckets of the normalized value n in [-1, 1]: u = RN(16 n + 16) in [0, 32].
+constexpr int kNumBuckets = 33;
+
+struct Nf4Tables {
+  float level[16];            // NF4 levels, ascending, level[7] == 0
+  float threshold[15];        // code(n) = #{i : n >= threshold[i]}
+  float bucket_thr[kNumBuckets];     // the one threshold inside bucket u, or +inf
+  uint8_t bucket_base[kNumBuckets];  // code of the smallest n in bucket u
+  bool ok;                    // every bucket holds at most one threshold
+};
+
+// Built once (thread-safe) on first use.
+const Nf4Tables& nf4_tables();
+
+}  // namespace qlora

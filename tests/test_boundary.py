@@ -1,0 +1,138 @@
+"""The C-ABI boundary on CPU: the library loads, exports every declared entry
+point, its host-side tables agree with the oracle, and argument validation
+rejects bad calls before anything reaches a GPU.  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qlora.h")
+
+qb = pytest.importorskip("bit_nf4_quantized_encode_b200")
+lib = qb._lib
+
+OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_UNSUP, ERR_CUDA, ERR_WS = 0, -1, -2, -3, -4, -5, -6
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"QLORA_EXPORT[^;(]*?\b(qlora_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_symbols()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in qlora.h but not exported"
+    assert set(names) == set(qb.EXPORTED)
+
+
+def test_codebook_matches_oracle_bit_for_bit():
+    ours = np.array(qb.qlora_get_codebook(), dtype=np.float32)
+    ref = oracle.codebook()
+    assert ours.view(np.uint32).tolist() == ref.view(np.uint32).tolist()
+
+
+@pytest.mark.parametrize("rows,cols", [(256, 256), (4096, 4096), (11008, 4096), (3, 100), (1, 1),
+                                       (0, 5), (22016, 8192)])
+def test_nf4_sizes_match_oracle(rows, cols):
+    sz = qb.qlora_nf4_sizes(rows, cols)
+    ref = oracle.storage_bytes(rows * cols)
+    assert sz["codes"] == ref["codes"]
+    assert sz["absmax_q"] == ref["absmax_q"]
+    assert sz["absmax_c2"] == ref["absmax_c2"]
+
+
+def _tensor(rows=64, cols=64, base=0x10000):
+    return qb._Nf4TensorC(base, base + 0x1000, base + 0x2000, base + 0x3000, rows, cols, 64, 256)
+
+
+def test_sizes_reject_bad_block_sizes_and_shapes():
+    z = ctypes.c_size_t()
+    assert lib.qlora_nf4_sizes(4, 64, 128, 256, None, None, None, ctypes.byref(z)) == ERR_UNSUP
+    assert lib.qlora_nf4_sizes(4, 64, 64, 512, None, None, None, None) == ERR_UNSUP
+    assert lib.qlora_nf4_sizes(-1, 64, 64, 256, None, None, None, None) == ERR_SHAPE
+
+
+def test_quantize_validation_before_launch():
+    t = _tensor()
+    w, ws = ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000)
+    assert lib.qlora_quantize_nf4_dq(None, ctypes.byref(t), ws, 1 << 20, None) == ERR_NULL
+    assert lib.qlora_quantize_nf4_dq(w, None, ws, 1 << 20, None) == ERR_NULL
+    assert lib.qlora_quantize_nf4_dq(ctypes.c_void_p(0x20008), ctypes.byref(t), ws, 1 << 20, None) == ERR_ALIGN
+    assert lib.qlora_quantize_nf4_dq(w, ctypes.byref(t), ws, 8, None) == ERR_WS
+    bad = _tensor()
+    bad.blocksize = 32
+    assert lib.qlora_quantize_nf4_dq(w, ctypes.byref(bad), ws, 1 << 20, None) == ERR_UNSUP
+    mis = _tensor()
+    mis.absmax_c2 = mis.absmax_c2 + 4
+    assert lib.qlora_quantize_nf4_dq(w, ctypes.byref(mis), ws, 1 << 20, None) == ERR_ALIGN
+    nul = _tensor()
+    nul.codes = None
+    assert lib.qlora_quantize_nf4_dq(w, ctypes.byref(nul), ws, 1 << 20, None) == ERR_NULL
+    empty = _tensor(rows=0)
+    assert lib.qlora_quantize_nf4_dq(None, ctypes.byref(empty), None, 0, None) == OK   # no-op
+
+
+def test_dequantize_validation_before_launch():
+    t = _tensor()
+    assert lib.qlora_dequantize(ctypes.byref(t), None, None) == ERR_NULL
+    assert lib.qlora_dequantize(ctypes.byref(t), ctypes.c_void_p(0x20002), None) == ERR_ALIGN
+
+
+def test_workspace_sizes():
+    f, b = qb.qlora_linear_workspace_size(4096, 4096, 8192, 64)
+    assert f >= 8192 * 64 * 6 and b >= (4096 + 4096) * 64 * 4
+    f16, b16 = qb.qlora_linear_workspace_size(22016, 8192, 16, 64)
+    assert f16 >= 16 * 22016 * 4            # split-K fp32 accumulator for decode shapes
+    with pytest.raises(qb.QloraError):
+        qb.qlora_linear_workspace_size(4096, 100, 16, 64)     # cols % 64 != 0
+    with pytest.raises(qb.QloraError):
+        qb.qlora_linear_workspace_size(4096, 4096, 16, 12)    # r % 8 != 0
+
+
+@pytest.mark.parametrize("rows,cols,m,r,expect", [
+    (4096, 4096, 0, 64, ERR_SHAPE),       # no tokens
+    (4096, 4100, 16, 64, ERR_SHAPE),      # cols not a multiple of 64 (tensor shape)
+    (4100, 4096, 16, 64, ERR_SHAPE),      # rows not a multiple of 8
+    (4096, 4096, 16, 4, ERR_SHAPE),       # rank below 8
+    (4096, 4096, 16, 264, ERR_SHAPE),     # rank above 256
+])
+def test_linear_shape_validation(rows, cols, m, r, expect):
+    t = _tensor(rows, cols)
+    p = ctypes.c_void_p(0x40000)
+    st = lib.qlora_linear_fwd(ctypes.byref(t), p, m, p, p, r, ctypes.c_float(0.25), p, None, p,
+                              1 << 40, None)
+    assert st == expect
+    st = lib.qlora_linear_bwd(ctypes.byref(t), p, p, m, p, p, r, ctypes.c_float(0.25), None, p, p, p,
+                              p, 1 << 40, None)
+    assert st == expect
+
+
+def test_linear_pointer_validation():
+    t = _tensor(256, 256)
+    p = ctypes.c_void_p(0x40000)
+    odd = ctypes.c_void_p(0x40002)
+    s = ctypes.c_float(2.0)
+    assert lib.qlora_linear_fwd(ctypes.byref(t), None, 16, p, p, 8, s, p, None, p, 1 << 40, None) == ERR_NULL
+    assert lib.qlora_linear_fwd(ctypes.byref(t), odd, 16, p, p, 8, s, p, None, p, 1 << 40, None) == ERR_ALIGN
+    assert lib.qlora_linear_fwd(ctypes.byref(t), p, 16, p, p, 8, s, p, odd, p, 1 << 40, None) == ERR_ALIGN
+    assert lib.qlora_linear_fwd(ctypes.byref(t), p, 16, p, p, 8, s, p, None, p, 16, None) == ERR_WS
+    assert lib.qlora_linear_fwd(ctypes.byref(t), p, 16, p, p, 8, ctypes.c_float(float("nan")), p, None,
+                                p, 1 << 40, None) == ERR_SHAPE
+    assert lib.qlora_linear_bwd(ctypes.byref(t), p, p, 16, p, p, 8, s, None, None, None, p, p,
+                                1 << 40, None) == ERR_NULL          # dA is required
+    assert lib.qlora_linear_bwd(ctypes.byref(t), p, p, 16, p, p, 8, s, odd, None, p, p, p,
+                                1 << 40, None) == ERR_ALIGN
+    assert lib.qlora_linear_bwd(ctypes.byref(t), p, p, 16, p, p, 8, s, None, None, p, p, p,
+                                64, None) == ERR_WS
+
+
+def test_status_strings():
+    for st in (OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_UNSUP, ERR_CUDA, ERR_WS, 12345):
+        assert isinstance(qb.qlora_status_string(st), str) and qb.qlora_status_string(st)

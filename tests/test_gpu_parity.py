@@ -1,0 +1,195 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.
+
+Bar: bit-exact for NF4 codes, E4M3 constants, c2, the mean and dequantized bf16
+weights; max |err| <= 2e-2 * rms(oracle) per tensor for Y, dX, dA, dB.
+The GEMM cases take the oracle's quantized weight as their input (uploaded),
+so they do not depend on the GPU encoder; every expected value comes from the
+oracle on the CPU.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+
+
+@pytest.fixture(scope="module")
+def qb():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import bit_nf4_quantized_encode_b200 as m
+    return m
+
+
+def _no_device_errors(qb):
+    torch.cuda.synchronize()
+    assert qb.qlora_read_device_errors() == 0
+
+
+def _upload_oracle_quant(qb, qt):
+    dev = torch.device("cuda")
+    t = qb.empty_nf4(qt["shape"][0] if len(qt["shape"]) == 2 else 1,
+                     qt["shape"][1] if len(qt["shape"]) == 2 else qt["numel"], dev)
+    t.codes[: qt["codes"].size].copy_(torch.from_numpy(qt["codes"]))
+    t.absmax_q[: qt["absmax_q"].size].copy_(torch.from_numpy(qt["absmax_q"]))
+    t.absmax_c2[: qt["absmax_c2"].size].copy_(torch.from_numpy(qt["absmax_c2"]))
+    t.absmax_mean[:1].copy_(torch.tensor([float(qt["mean"])], dtype=torch.float32))
+    return t
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16).reshape(-1)
+
+
+def _assert_codec_equal(qb, w_cpu: torch.Tensor):
+    bits = workloads.bf16_bits(w_cpu)
+    ref = oracle.quantize(bits)
+    got = qb.qlora_quantize_nf4_dq(w_cpu.cuda())
+    _no_device_errors(qb)
+    n = ref["codes"].size
+    codes = got.codes[:n].cpu().numpy()
+    bad = np.nonzero(codes != ref["codes"])[0]
+    assert bad.size == 0, f"{bad.size} code bytes differ; first at byte {bad[0]}: {codes[bad[0]]:#x} vs {ref['codes'][bad[0]]:#x}"
+    nb = ref["absmax_q"].size
+    assert np.array_equal(got.absmax_mean[:1].cpu().numpy().view(np.uint32),
+                          np.array([ref["mean"]], np.float32).view(np.uint32))
+    assert np.array_equal(got.absmax_c2[: ref["absmax_c2"].size].cpu().numpy().view(np.uint32),
+                          ref["absmax_c2"].view(np.uint32))
+    assert np.array_equal(got.absmax_q[:nb].cpu().numpy(), ref["absmax_q"])
+    # dequantize the ORACLE's stored tensor on the GPU and compare with the oracle's dequant
+    up = _upload_oracle_quant(qb, ref)
+    deq = qb.qlora_dequantize(up)
+    _no_device_errors(qb)
+    ref_deq = oracle.dequant(ref["codes"], ref["absmax_q"], ref["absmax_c2"], ref["mean"], ref["numel"])
+    got_deq = _bits(deq)[: ref["numel"]]
+    bad = np.nonzero(got_deq != ref_deq)[0]
+    assert bad.size == 0, f"{bad.size} dequantized weights differ; first {bad[0]}"
+
+
+@pytest.mark.parametrize("shape", [(256, 256), (64, 64), (128, 192), (3, 100), (1, 1), (1, 7),
+                                   (5, 13), (1, 64 * 256 + 8), (300, 4160)])
+def test_codec_small_and_ragged(qb, shape):
+    w = workloads.weight(shape, proj=shape[0] % 7)
+    _assert_codec_equal(qb, w)
+
+
+def test_codec_4096_outliers(qb):
+    w = workloads.weight((4096, 4096), proj=0, outliers=True)
+    _assert_codec_equal(qb, w)
+
+
+@pytest.mark.parametrize("shape", [(11008, 4096), (22016, 8192)])
+def test_codec_llama_shapes(qb, shape):
+    _assert_codec_equal(qb, workloads.weight(shape, proj=4))
+
+
+def test_codec_thresholds_and_levels(qb):
+    """Weights placed at, just above and just below every decision midpoint, and
+    at every level, with block absmax 1 so the quotient is the value itself."""
+    L = oracle.codebook()
+    vals = []
+    for i in range(15):
+        m = np.float32((float(L[i]) + float(L[i + 1])) / 2)
+        vals += [m, np.nextafter(m, np.float32(2)), np.nextafter(m, np.float32(-2))]
+    vals += list(L)
+    vals = oracle.bf16_bits_to_f32(oracle.bf16_rne_array(np.array(vals, np.float32)))
+    blocks = []
+    for i in range(0, len(vals), 62):
+        chunk = list(vals[i:i + 62]) + [1.0, -1.0]
+        blocks += chunk + [0.0] * (64 - len(chunk))
+    # scaled copies exercise other absmax values with the same quotients
+    base = np.array(blocks, np.float32)
+    allw = np.concatenate([base * np.float32(s) for s in (1.0, 0.5, 0.0078125, 3.0)])
+    w = torch.from_numpy(allw).to(torch.bfloat16).reshape(1, -1)
+    _assert_codec_equal(qb, w)
+
+
+def test_codec_zero_and_constant_blocks(qb):
+    w = torch.zeros(4, 512, dtype=torch.bfloat16)
+    w[1, :] = 0.5                      # constant blocks: c2 may be zero in a group
+    w[2, 64:128] = -0.25
+    _assert_codec_equal(qb, w)
+
+
+# ------------------------------------------------------------------ linear layer
+def _linear_case(qb, n, k, m, r, alpha, proj, rows_sample=None, check_bwd=True, with_xa=True):
+    w = workloads.weight((n, k), proj=proj)
+    qt = oracle.quantize(workloads.bf16_bits(w))
+    Wd = oracle.dequant_tensor(qt)                      # float32 [n, k], bf16-exact
+    X = workloads.activations(m, k, proj)
+    A = workloads.lora_a(r, k, proj)
+    B = workloads.lora_b(n, r, proj)
+    dY = workloads.grad_output(m, n, proj)
+    s = alpha / r
+    up = _upload_oracle_quant(qb, qt)
+    Xg, Ag, Bg, dYg = X.cuda(), A.cuda(), B.cuda(), dY.cuda()
+    Y, XA = qb.qlora_linear_fwd(up, Xg, Ag, Bg, s, save_xa=True)
+    _no_device_errors(qb)
+    rows = np.arange(m) if rows_sample is None else rows_sample
+    Xf, Af, Bf, dYf = (t.float().numpy() for t in (X, A, B, dY))
+    Y_ref = oracle.linear_fwd_rows(Wd, Xf, Af, Bf, s, rows)
+    _close("Y", Y.float().cpu().numpy()[rows], Y_ref)
+    XA_ref = Xf[rows].astype(np.float64) @ Af.T.astype(np.float64)
+    _close("XA", XA.float().cpu().numpy()[rows], XA_ref)
+    if not check_bwd:
+        return
+    dX, dA, dB = qb.qlora_linear_bwd(up, Xg, dYg, Ag, Bg, s, XA=XA if with_xa else None)
+    _no_device_errors(qb)
+    dX_ref = oracle.linear_bwd_dx_rows(Wd, dYf, Af, Bf, s, rows)
+    _close("dX", dX.float().cpu().numpy()[rows], dX_ref)
+    XAf = Xf.astype(np.float64) @ Af.T.astype(np.float64)
+    G = dYf.astype(np.float64) @ Bf.astype(np.float64)
+    dB_ref = s * (dYf.T.astype(np.float64) @ XAf)
+    dA_ref = s * (G.T @ Xf.astype(np.float64))
+    _close("dA", dA.float().cpu().numpy(), dA_ref)
+    _close("dB", dB.float().cpu().numpy(), dB_ref)
+
+
+def _close(name, got, ref):
+    ref = np.asarray(ref, np.float64)
+    got = np.asarray(got, np.float64)
+    assert got.shape == ref.shape, (name, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{name}: non-finite output"
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    err = float(np.max(np.abs(got - ref)))
+    assert err <= TOL * rms, f"{name}: max|err| {err:.4g} > {TOL} * rms {rms:.4g} (ratio {err / rms:.4g})"
+
+
+def test_linear_tiny_layer(qb):
+    """The 256x256 layer, 16 tokens, r = 8, alpha = 16 (s = 2): forward and backward."""
+    _linear_case(qb, 256, 256, 16, 8, 16.0, proj=0)
+
+
+@pytest.mark.parametrize("m", [1, 4, 16])
+def test_linear_decode_shapes(qb, m):
+    _linear_case(qb, 392, 640, m, 64, 16.0, proj=1)
+
+
+@pytest.mark.parametrize("n,k,m,r", [(392, 320, 300, 16), (256, 512, 257, 64), (136, 192, 520, 72),
+                                     (512, 256, 1024, 128)])
+def test_linear_prefill_ragged(qb, n, k, m, r):
+    _linear_case(qb, n, k, m, r, 16.0, proj=2)
+
+
+def test_linear_bwd_recomputes_xa(qb):
+    _linear_case(qb, 264, 384, 96, 64, 16.0, proj=3, with_xa=False)
+
+
+def test_linear_llama7b_q_projection_full_size(qb):
+    """4096 x 4096 at 8192 tokens (r = 64): Y and dX on 256 sampled token rows,
+    dA and dB in full."""
+    rng = np.random.Generator(np.random.PCG64(99))
+    rows = np.sort(rng.choice(8192, 256, replace=False))
+    _linear_case(qb, 4096, 4096, 8192, 64, 16.0, proj=0, rows_sample=rows)
+
+
+def test_linear_gemv_65b_ffn(qb):
+    """22016 x 8192 and 8192 x 22016 at 16 tokens, forward (decode-shaped GEMV)."""
+    _linear_case(qb, 22016, 8192, 16, 64, 16.0, proj=5, check_bwd=False)
+    _linear_case(qb, 8192, 22016, 4, 64, 16.0, proj=6, check_bwd=False)
