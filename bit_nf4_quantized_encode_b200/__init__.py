@@ -64,6 +64,8 @@ _lib.qlora_linear_bwd.argtypes = [_T, _vp, _vp, _i64, _vp, _vp, _i32, ctypes.c_f
 _lib.qlora_linear_bwd.restype = ctypes.c_int
 _lib.qlora_read_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
 _lib.qlora_read_device_errors.restype = ctypes.c_int
+_lib.qlora_quantize_nf4_dq_noalloc.argtypes = [_vp, _T, _vp]
+_lib.qlora_quantize_nf4_dq_noalloc.restype = ctypes.c_int
 _lib.qlora_kernel_launches.argtypes = []
 _lib.qlora_kernel_launches.restype = ctypes.c_uint64
 _lib.qlora_time_next_gemm.argtypes = [_vp, _vp]
@@ -72,7 +74,10 @@ _lib.qlora_time_next_gemm.restype = ctypes.c_int
 EXPORTED = ["qlora_status_string", "qlora_get_codebook", "qlora_nf4_sizes", "qlora_quantize_nf4_dq",
             "qlora_dequantize", "qlora_linear_workspace_size", "qlora_linear_fwd",
             "qlora_linear_bwd", "qlora_read_device_errors", "qlora_kernel_launches",
-            "qlora_time_next_gemm"]
+            "qlora_time_next_gemm", "qlora_quantize_nf4_dq_noalloc"]
+
+# Largest weight the allocation-free quantize variant accepts.
+NOALLOC_MAX_ELEMENTS = 134217728
 
 
 class QloraError(RuntimeError):
@@ -165,6 +170,16 @@ def qlora_quantize_nf4_dq(W: torch.Tensor, out: NF4Tensor | None = None,
     c = out.c_struct()
     _check(_lib.qlora_quantize_nf4_dq(_ptr(W), ctypes.byref(c), _ptr(workspace),
                                       workspace.numel(), _stream(W.device)), "qlora_quantize_nf4_dq")
+    return out
+
+
+def qlora_quantize_nf4_dq_noalloc(W: torch.Tensor, out: NF4Tensor) -> NF4Tensor:
+    """Same result as qlora_quantize_nf4_dq, with the library's built-in scratch
+    instead of a work buffer (for callers that cannot allocate; see qlora.h)."""
+    _need_bf16_cuda("W", W)
+    c = out.c_struct()
+    _check(_lib.qlora_quantize_nf4_dq_noalloc(_ptr(W), ctypes.byref(c), _stream(W.device)),
+           "qlora_quantize_nf4_dq_noalloc")
     return out
 
 

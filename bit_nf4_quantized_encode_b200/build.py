@@ -14,7 +14,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libqlora.so")
-SOURCES = ["api.cu", "codec.cu", "gemm.cu", "nf4_tables.cpp"]
+SOURCES = ["api.cu", "codec.cu", "gemm.cu", "noalloc.cu", "nf4_tables.cpp"]
 HEADERS = ["codec.h", "gemm.h", "nf4_device.cuh", "nf4_tables.h", "sm100_ptx.cuh"]
 
 

@@ -174,6 +174,33 @@ QLORA_EXPORT qlora_status qlora_linear_bwd(const qlora_nf4_tensor* W, const uint
 QLORA_EXPORT qlora_status qlora_read_device_errors(uint32_t* flags, int clear);
 
 /*
+ * Largest weight (rows * cols) qlora_quantize_nf4_dq_noalloc accepts.
+ */
+#define QLORA_NOALLOC_MAX_ELEMENTS 134217728LL   /* 2^27, e.g. 8192 x 16384 */
+
+/*
+ * qlora_quantize_nf4_dq without a work buffer and without any allocation.
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot obtain device memory when they quantize: a server that reserves
+ * all of its memory at start-up and forbids allocation afterwards, code that
+ * runs inside another framework's allocator or out-of-memory path, or a loader
+ * with no allocator handle.  Its scratch (one float per 64 weights plus 2048
+ * partial sums, 8 MiB + 16 KiB) is a fixed array inside the library that
+ * every GPU loading the library holds until the process exits.
+ *   - Same arguments and results as qlora_quantize_nf4_dq, bit for bit.
+ *   - rows * cols above QLORA_NOALLOC_MAX_ELEMENTS: QLORA_ERR_WORKSPACE,
+ *     nothing launched.  Other validation as for qlora_quantize_nf4_dq.
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address; make that first call before any stream capture.
+ *   - All calls share the one array: calls that can overlap on the GPU (other
+ *     streams, other host threads) race on it and must be ordered by the
+ *     caller.  No part of the array needs clearing between calls.
+ *   - Calls no cudaMalloc / cudaFree or other allocating routine.
+ */
+QLORA_EXPORT qlora_status qlora_quantize_nf4_dq_noalloc(const uint16_t* W, const qlora_nf4_tensor* out,
+                                                     qlora_stream_t stream);
+
+/*
  * Number of kernels this library has launched in the process so far (all
  * devices).  Host only; used to count launches inside a timed region.
  */
