@@ -444,6 +444,43 @@ def bench_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_case(args):
+    """One operation on a small case, for profiler captures (prints timings, no JSON)."""
+    import torch
+    import bit_nf4_quantized_encode_b200 as qb
+    device = torch.device("cuda", 0)
+    n, k, m, r = args.case_n, args.case_k, args.case_m, 64
+    w = workloads.weight((n, k), proj=0).to(device)
+    qt = qb.qlora_quantize_nf4_dq(w)
+    X = workloads.activations(m, k).to(device)
+    dY = workloads.grad_output(m, n).to(device)
+    A, B = workloads.lora_a(r, k).to(device), workloads.lora_b(n, r).to(device)
+    fw, bw = qb.qlora_linear_workspace_size(n, k, m, r)
+    wsf = torch.empty(fw, dtype=torch.uint8, device=device)
+    wsb = torch.empty(bw, dtype=torch.uint8, device=device)
+    Y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+    XA = torch.empty(m, r, dtype=torch.float32, device=device)
+    out = torch.empty(n, k, dtype=torch.bfloat16, device=device)
+    wse = torch.empty(qb.qlora_nf4_sizes(n, k)["workspace"], dtype=torch.uint8, device=device)
+    ops = {
+        "fused_fwd": lambda: qb.qlora_linear_fwd(qt, X, A, B, 0.25, Y=Y, XA=XA, workspace=wsf),
+        "fused_bwd": lambda: qb.qlora_linear_bwd(qt, X, dY, A, B, 0.25, XA=XA, workspace=wsb),
+        "encode": lambda: qb.qlora_quantize_nf4_dq(w, out=qt, workspace=wse),
+        "dequant": lambda: qb.qlora_dequantize(qt, out=out),
+    }
+    fn = ops[args.case]
+    qb.qlora_linear_fwd(qt, X, A, B, 0.25, Y=Y, XA=XA, workspace=wsf)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.case_iters):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    assert qb.qlora_read_device_errors() == 0
+    print(f"case {args.case} n={n} k={k} m={m}: {e0.elapsed_time(e1) / args.case_iters * 1e3:.1f} us/call")
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -454,7 +491,16 @@ def main():
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=64, help="token sample of the CPU-oracle baseline")
     ap.add_argument("--ref-tokens", type=int, default=16, help="token sample per reference-arm step")
+    ap.add_argument("--case", choices=["fused_fwd", "fused_bwd", "encode", "dequant"],
+                    help="run one operation on a small case (for profiler captures) and exit")
+    ap.add_argument("--case-n", type=int, default=8192)
+    ap.add_argument("--case-k", type=int, default=8192)
+    ap.add_argument("--case-m", type=int, default=4096)
+    ap.add_argument("--case-iters", type=int, default=3)
     args = ap.parse_args()
+    if args.case:
+        run_case(args)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

@@ -27,13 +27,15 @@ namespace qlora {
 namespace {
 
 constexpr int kATileBytes = 128 * 128;     // 128 rows x 64 bf16, 128B-swizzled
-constexpr int kNumDequantWarps = 8;        // two groups of 128 threads, alternating k-steps
-constexpr int kEpiWarp0 = 8;               // warps 8..11: epilogue (TMEM lane quarters 0..3)
-constexpr int kTmaWarp = 12;
-constexpr int kMmaWarp = 13;
-constexpr int kFusedThreads = 14 * 32;
+constexpr int kDequantGroups = 4;          // groups of 128 threads; group g takes k-steps = g mod 4
+constexpr int kNumDequantWarps = 4 * kDequantGroups;
+constexpr int kEpiWarp0 = kNumDequantWarps;          // 4 epilogue warps (TMEM lane quarters 0..3)
+constexpr int kTmaWarp = kEpiWarp0 + 4;
+constexpr int kMmaWarp = kTmaWarp + 1;
+constexpr int kFusedThreads = (kMmaWarp + 1) * 32;
 
 __host__ __device__ constexpr int fused_stages(int bn) { return bn >= 128 ? 4 : 8; }
+static_assert(kDequantGroups == 4, "stage ring and group rotation assume four groups");
 __host__ __device__ constexpr int fused_tmem_cols(int bn) { return 2 * bn < 32 ? 32 : 2 * bn; }
 __host__ __device__ constexpr size_t fused_smem_bytes(int bn) {
   return 1024 + static_cast<size_t>(fused_stages(bn)) * (kATileBytes + bn * 128) + 512;
@@ -213,7 +215,7 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
 
   if (warp < kNumDequantWarps) {
     // ------------------------------------------------ dequant producers
-    const int group = warp >> 2;              // 0: warps 0-3, 1: warps 4-7
+    const int group = warp >> 2;              // warps 4g .. 4g+3
     const int t = threadIdx.x & 127;
     const float mu = __ldg(a.mean);
     uint32_t gctr = 0;
@@ -221,14 +223,14 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
     for (int u = blockIdx.x; u < nunits && alive; u += gridDim.x) {
       const Unit w = decode_unit(u, a.m_tiles, a.splits, a.ksteps, a.lora_steps);
       const int m0 = w.mt * 128;
-      int j = static_cast<int>((static_cast<uint32_t>(group) - gctr) & 1u);
+      int j = static_cast<int>((static_cast<uint32_t>(group) - gctr) & (kDequantGroups - 1));
       DqLoad next;
       if (j < w.kmain) next = dq_load<kDir>(a, m0, w.kbeg + j, t);
-      for (; j < w.nk; j += 2) {
+      for (; j < w.nk; j += kDequantGroups) {
         const uint32_t it = gctr + j;
         const uint32_t stage = it % kStages, phase = (it / kStages) & 1u;
         const DqLoad cur = next;
-        if (j + 2 < w.kmain) next = dq_load<kDir>(a, m0, w.kbeg + j + 2, t);
+        if (j + kDequantGroups < w.kmain) next = dq_load<kDir>(a, m0, w.kbeg + j + kDequantGroups, t);
         if (!mbar_wait(&empty[stage], phase ^ 1u, a.err)) { alive = false; break; }
         const uint32_t sA = smem0 + stage * kStageBytes;
         if (j < w.kmain) dq_store<kDir>(sA, t, cur, mu, a.cb);
@@ -295,7 +297,7 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
     }
   } else {
     // ------------------------------------------------ epilogue: TMEM -> global
-    const int quarter = warp & 3;             // warps 8..11 -> lane quarters 0..3
+    const int quarter = warp & 3;             // the four epilogue warps cover lane quarters 0..3
     uint32_t uctr = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++uctr) {
       const Unit w = decode_unit(u, a.m_tiles, a.splits, a.ksteps, a.lora_steps);
