@@ -14,6 +14,7 @@
 
 #include "codec.h"
 #include "gemm.h"
+#include "gemv.h"
 #include "nf4_tables.h"
 #include "qlora.h"
 
@@ -107,6 +108,34 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
   return r == CUDA_SUCCESS;
 }
 
+// 2-D uint8 tensor map without swizzle (packed NF4 codes): dims {inner, outer}.
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch_bytes,
+                 uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {pitch_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Split count for `tiles` output tiles of `ksteps` steps each over `sms` CTAs:
+// minimises the makespan ceil(tiles * s / sms) * ceil(ksteps / s), counting two
+// steps of fixed cost per work unit.
+int balanced_splits(int tiles, int ksteps, int sms) {
+  int best = 1;
+  int64_t best_cost = -1;
+  for (int s = 1; s <= ksteps && s <= 128; ++s) {
+    const int64_t waves = (static_cast<int64_t>(tiles) * s + sms - 1) / sms;
+    const int64_t cost = waves * ((ksteps + s - 1) / s + 2);
+    if (best_cost < 0 || cost < best_cost) { best_cost = cost; best = s; }
+  }
+  return best;
+}
+
 qlora_status check_tensor(const qlora_nf4_tensor* t) {
   if (!t) return QLORA_ERR_NULL;
   if (t->rows < 0 || t->cols < 0 || t->rows > kMaxDim || t->cols > kMaxDim) return QLORA_ERR_SHAPE;
@@ -154,13 +183,20 @@ qlora_status check_linear(const qlora_nf4_tensor* W, int64_t M, int32_t r, Linea
 // Work buffer layout: fp32 accumulators first (one memset clears them all),
 // then bf16 staging.  Offsets in bytes, each 256-aligned.
 struct FwdLayout {
-  size_t xa_acc, y_acc, fp32_end, sxa, total;
+  size_t xa_acc, y_acc, fp32_end, sxa, xa_part, counters, total;
 };
 FwdLayout fwd_layout(const LinearShape& s) {
   FwdLayout l{};
   size_t o = 0;
+  if (s.decode) {        // k_xa_small + k_gemv: X A^T, split buffer, tile counters
+    l.y_acc = o;    o = round_up(o + size_t(s.m) * s.rows * 4, 256);
+    l.xa_part = o;  o = round_up(o + size_t(16) * s.rpad * 4, 256);
+    l.counters = o; o = round_up(o + size_t((s.rows + gemv_tile_rows() - 1) / gemv_tile_rows()) * 4, 256);
+    l.fp32_end = 0;
+    l.total = o;
+    return l;
+  }
   l.xa_acc = o; o = round_up(o + size_t(s.m) * s.rpad * 4, 256);
-  l.y_acc = o;  if (s.decode) o = round_up(o + size_t(s.m) * s.rows * 4, 256);
   l.fp32_end = o;
   l.sxa = o;    o = round_up(o + size_t(s.m) * s.rpad * 2, 256);
   l.total = o;
@@ -345,10 +381,39 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor* W, const uint16_t* X, int6
   if ((st = device_info(&d)) != QLORA_OK) return st;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* xa_acc = reinterpret_cast<float*>(ws + L.xa_acc);
-  float* y_acc = reinterpret_cast<float*>(ws + L.y_acc);
-  uint16_t* sxa = reinterpret_cast<uint16_t*>(ws + L.sxa);
 
+  if (sh.decode) {
+    // Decode shapes: X A^T partials (k_xa_small, which also zeroes the split-K
+    // buffer and tile counters), then one pass over the packed weight (k_gemv).
+    float* y_acc = reinterpret_cast<float*>(ws + L.y_acc);
+    float* xa = reinterpret_cast<float*>(ws + L.xa_part);
+    int* counters = reinterpret_cast<int*>(ws + L.counters);
+    const int m_tiles = static_cast<int>((sh.rows + gemv_tile_rows() - 1) / gemv_tile_rows());
+    if (counted(launch_xa_small(X, A, sh.m, sh.cols, sh.r, xa, sh.rpad, XA_out, y_acc, sh.m * sh.rows,
+                                counters, m_tiles, cs)) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    CUtensorMap c_map, x_act;
+    if (!make_map_u8(&c_map, W->codes, sh.cols / 2, sh.rows, sh.cols / 2, 128, gemv_tile_rows(),
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&x_act, X, sh.cols, sh.m, sh.cols * 2, 16))
+      return QLORA_ERR_CUDA;
+    GemvArgs ga{};
+    ga.qabs = W->absmax_q; ga.c2 = W->absmax_c2; ga.mean = W->absmax_mean;
+    ga.nw = sh.rows; ga.kw = sh.cols; ga.m = sh.m;
+    ga.yacc = y_acc; ga.counters = counters;
+    ga.xa = xa; ga.ld_xa = sh.rpad;
+    ga.lora_b = B; ga.r = sh.r; ga.s = s; ga.y = Y;
+    ga.m_tiles = m_tiles;
+    ga.steps = static_cast<int>((sh.cols / 64 + 3) / 4);
+    const CodebookParam cbp = codebook_param();
+    for (int i = 0; i < 16; ++i) ga.level[i] = cbp.level[i];
+    ga.err = d.err;
+    if (counted(launch_gemv(ga, c_map, x_act, d.num_sms, cs)) != cudaSuccess) return QLORA_ERR_CUDA;
+    return QLORA_OK;
+  }
+
+  float* xa_acc = reinterpret_cast<float*>(ws + L.xa_acc);
+  uint16_t* sxa = reinterpret_cast<uint16_t*>(ws + L.sxa);
   if (cudaMemsetAsync(ws, 0, L.fp32_end, cs) != cudaSuccess) return QLORA_ERR_CUDA;
 
   // 1) XA = X A^T  (skinny tcgen05 GEMM, split-K into fp32)
@@ -382,15 +447,11 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor* W, const uint16_t* X, int6
   fa.ksteps = static_cast<int>(sh.cols / 64);
   fa.m_tiles = static_cast<int>((sh.rows + 127) / 128);
   fa.t_tiles = static_cast<int>((sh.m + bn - 1) / bn);
-  fa.splits = sh.decode ? choose_splits(fa.m_tiles, fa.ksteps, d.num_sms) : 1;
-  fa.out = Y; fa.out_acc = y_acc;
+  fa.splits = 1;
+  fa.out = Y; fa.out_acc = nullptr;
   fa.cb = codebook_param();
   fa.err = d.err;
   if (fused_timed(FusedDir::kFwd, bn, fa, x_act, sxa_map, d.num_sms, cs) != cudaSuccess)
-    return QLORA_ERR_CUDA;
-  if (fa.splits > 1 &&
-      counted(launch_convert_bf16(y_acc, sh.m, sh.rows, sh.rows, sh.rows, 1.0f, Y, sh.rows, cs)) !=
-          cudaSuccess)
     return QLORA_ERR_CUDA;
   return QLORA_OK;
 }
