@@ -183,15 +183,14 @@ qlora_status check_linear(const qlora_nf4_tensor* W, int64_t M, int32_t r, Linea
 // Work buffer layout: fp32 accumulators first (one memset clears them all),
 // then bf16 staging.  Offsets in bytes, each 256-aligned.
 struct FwdLayout {
-  size_t xa_acc, y_acc, fp32_end, sxa, xa_part, counters, total;
+  size_t xa_acc, y_acc, fp32_end, sxa, xa_part, total;
 };
 FwdLayout fwd_layout(const LinearShape& s) {
   FwdLayout l{};
   size_t o = 0;
-  if (s.decode) {        // k_xa_small + k_gemv: X A^T, split buffer, tile counters
+  if (s.decode) {        // k_gemv_zero + k_gemv + k_finish: split buffer, X A^T
     l.y_acc = o;    o = round_up(o + size_t(s.m) * s.rows * 4, 256);
     l.xa_part = o;  o = round_up(o + size_t(16) * s.rpad * 4, 256);
-    l.counters = o; o = round_up(o + size_t((s.rows + gemv_tile_rows() - 1) / gemv_tile_rows()) * 4, 256);
     l.fp32_end = 0;
     l.total = o;
     return l;
@@ -308,6 +307,8 @@ qlora_status qlora_quantize_nf4_dq(const uint16_t* W, const qlora_nf4_tensor* ou
     et.bucket_thr[i] = i < kNumBuckets ? tabs.bucket_thr[i] : INFINITY;
     et.bucket_base[i] = i < kNumBuckets ? tabs.bucket_base[i] : 15;
   }
+  et.fast = tabs.fast_ok ? 1 : 0;
+
   const int64_t nblocks = (numel + kBlock - 1) / kBlock;
   float* c1buf = static_cast<float*>(workspace);
   double* partials = reinterpret_cast<double*>(static_cast<uint8_t*>(workspace) +
@@ -383,32 +384,32 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor* W, const uint16_t* X, int6
   uint8_t* ws = static_cast<uint8_t*>(workspace);
 
   if (sh.decode) {
-    // Decode shapes: X A^T partials (k_xa_small, which also zeroes the split-K
-    // buffer and tile counters), then one pass over the packed weight (k_gemv).
+    // Decode shapes: zeroed accumulators (k_gemv_zero), one pass over the
+    // packed weight that also forms X A^T (k_gemv), then Y with the LoRA term
+    // (k_finish); each kernel is the programmatic dependent of the one before.
     float* y_acc = reinterpret_cast<float*>(ws + L.y_acc);
     float* xa = reinterpret_cast<float*>(ws + L.xa_part);
-    int* counters = reinterpret_cast<int*>(ws + L.counters);
     const int m_tiles = static_cast<int>((sh.rows + gemv_tile_rows() - 1) / gemv_tile_rows());
-    if (counted(launch_xa_small(X, A, sh.m, sh.cols, sh.r, xa, sh.rpad, XA_out, y_acc, sh.m * sh.rows,
-                                counters, m_tiles, cs)) != cudaSuccess)
+    if (counted(launch_gemv_zero(y_acc, sh.m * sh.rows, xa, 16 * sh.rpad, cs)) != cudaSuccess)
       return QLORA_ERR_CUDA;
     CUtensorMap c_map, x_act;
     if (!make_map_u8(&c_map, W->codes, sh.cols / 2, sh.rows, sh.cols / 2, 128, gemv_tile_rows(),
                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&x_act, X, sh.cols, sh.m, sh.cols * 2, 16))
+        !make_map(&x_act, X, sh.cols, sh.m, sh.cols * 2, static_cast<uint32_t>(sh.m)))
       return QLORA_ERR_CUDA;
     GemvArgs ga{};
     ga.qabs = W->absmax_q; ga.c2 = W->absmax_c2; ga.mean = W->absmax_mean;
     ga.nw = sh.rows; ga.kw = sh.cols; ga.m = sh.m;
-    ga.yacc = y_acc; ga.counters = counters;
-    ga.xa = xa; ga.ld_xa = sh.rpad;
-    ga.lora_b = B; ga.r = sh.r; ga.s = s; ga.y = Y;
+    ga.yacc = y_acc;
+    ga.x = X; ga.lora_a = A; ga.xa = xa; ga.ld_xa = sh.rpad; ga.r = sh.r;
     ga.m_tiles = m_tiles;
     ga.steps = static_cast<int>((sh.cols / 64 + 3) / 4);
     const CodebookParam cbp = codebook_param();
     for (int i = 0; i < 16; ++i) ga.level[i] = cbp.level[i];
     ga.err = d.err;
     if (counted(launch_gemv(ga, c_map, x_act, d.num_sms, cs)) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (counted(launch_gemv_finish(y_acc, xa, sh.rpad, B, sh.r, s, sh.m, sh.rows, Y, XA_out, cs)) != cudaSuccess)
+      return QLORA_ERR_CUDA;
     return QLORA_OK;
   }
 

@@ -33,7 +33,7 @@ namespace qlora {
 enum : int { kVecNone = 0, kVecFull = 1, kVecTail = 2 };
 
 __device__ __forceinline__ void encode_vec(const uint16_t* __restrict__ w, int64_t numel,
-                                           int64_t v, int mode, const float* s_thr,
+                                           int64_t v, int mode, bool fast, const float* s_thr,
                                            const uint8_t* s_base, uint8_t* __restrict__ codes,
                                            float* __restrict__ c1buf, double& csum) {
   float x[8];
@@ -59,16 +59,42 @@ __device__ __forceinline__ void encode_vec(const uint16_t* __restrict__ w, int64
 
   uint32_t packed = 0x77777777u;          // all zero-level codes
   if (amax > 0.0f) {
-    packed = 0;
+    // Fast path: n' = RN(x * RN(1/c1)) is within 2^-22 of the IEEE quotient
+    // RN(x / c1) (three roundings of relative size 2^-24, |n| <= 1), so its
+    // code equals the quotient's unless a threshold lies within 2^-22 of n'.
+    // The bucket of n' holds the only threshold that close (the table check
+    // keeps every threshold 2^-20 away from bucket edges); when n' is within
+    // 2^-20 of it the block's vector is redone with IEEE divisions.
+    bool exact = !fast || amax < 0x1.0p-125f;       // 1 / c1 must stay finite
+    if (!exact) {
+      const float r = __frcp_rn(amax);
+      uint32_t pk = 0;
+      bool risky = false;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float n = __fdiv_rn(x[i], amax);
-      // bucket u = RN(16 n + 16) via one fma against 2^23; then one compare
-      const uint32_t u = __float_as_uint(__fmaf_rn(n, 16.0f, 8388624.0f)) & 63u;
-      uint32_t code = s_base[u] + (n >= s_thr[u] ? 1u : 0u);
-      if (mode == kVecTail && e0 + i >= numel) code = 7u;
-      // element 2j -> high nibble of byte j, element 2j+1 -> low nibble
-      packed |= code << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
+      for (int i = 0; i < 8; ++i) {
+        const float n = __fmul_rn(x[i], r);
+        const uint32_t u = __float_as_uint(__fmaf_rn(n, 16.0f, 8388624.0f)) & 63u;
+        const float d = __fsub_rn(n, s_thr[u]);     // exact sign; -inf when the bucket has no threshold
+        uint32_t code = s_base[u] + (d >= 0.0f ? 1u : 0u);
+        risky |= fabsf(d) <= 0x1.0p-20f;
+        if (mode == kVecTail && e0 + i >= numel) code = 7u;
+        pk |= code << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
+      }
+      if (risky) exact = true;
+      else packed = pk;
+    }
+    if (exact) {
+      packed = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float n = __fdiv_rn(x[i], amax);
+        // bucket u = RN(16 n + 16) via one fma against 2^23; then one compare
+        const uint32_t u = __float_as_uint(__fmaf_rn(n, 16.0f, 8388624.0f)) & 63u;
+        uint32_t code = s_base[u] + (n >= s_thr[u] ? 1u : 0u);
+        if (mode == kVecTail && e0 + i >= numel) code = 7u;
+        // element 2j -> high nibble of byte j, element 2j+1 -> low nibble
+        packed |= code << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
+      }
     }
   }
   if (mode == kVecFull) {
@@ -109,7 +135,7 @@ __global__ void __launch_bounds__(256) k_encode(const uint16_t* __restrict__ w, 
     const int64_t v = base + threadIdx.x;
     const int64_t blk = v >> 3;                     // the same for all 8 lanes of a group
     const int mode = (blk < full_blocks) ? kVecFull : (blk < nblocks ? kVecTail : kVecNone);
-    encode_vec(w, numel, v, mode, s_thr, s_base, codes, c1buf, csum);
+    encode_vec(w, numel, v, mode, tab.fast != 0, s_thr, s_base, codes, c1buf, csum);
   }
   // deterministic per-CTA reduction of the partial sums
 #pragma unroll

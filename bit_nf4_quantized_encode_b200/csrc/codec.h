@@ -12,6 +12,7 @@ constexpr int kBuckets = 64;
 struct EncodeTables {
   float bucket_thr[kBuckets];
   uint8_t bucket_base[kBuckets];
+  int fast;                  // nonzero: the reciprocal path of the encoder may be used
 };
 
 // The 16 NF4 levels, passed by value.

@@ -2,29 +2,34 @@
 //
 // Y = X deq(W)^T + s (X A^T) B^T with few token rows is a stream over the packed
 // weight (automatone "QLoRA paper explained", section "How it works": the 4-bit
-// weight is dequantized on the fly for the matmul), bound by HBM.  Two kernels:
+// weight is dequantized on the fly for the matmul), bound by HBM.  Three
+// kernels, each launched as the programmatic dependent of the one before it:
 //
-// k_xa_small: X A^T in fp32 on CUDA cores (one CTA per LoRA rank column); also
-//   zeroes the split buffer and tile counters of k_gemv.
+// k_gemv_zero: zeroes the fp32 accumulators of k_gemv (split buffer, X A^T).
 //
 // k_gemv: the weight stream.  Each CTA takes an equal, contiguous share of all
 //   (256-row tile, 256-column step) pairs, so the work is balanced whatever the
-//   shape (a tile split between CTAs is combined with fp32 atomics).
-//   * A TMA warp streams the [256 rows x 128 bytes] code tile (128B-swizzled)
-//     and the four [16 x 64] activation boxes of each step into a 3-deep ring.
-//   * Sixteen warps own 16 weight rows each.  For every 64-column block they read
-//     the rows' 32 code bytes, turn each byte into the two bf16 levels it
-//     encodes with one shared-memory load from a 256-entry pair table (one copy
-//     per lane: conflict-free), and feed them straight from registers to warp
-//     MMAs (m16n8k16, bf16 in, fp32 out): a code byte is exactly one A-fragment
-//     register.  The block's product is scaled by its constant
+//   shape; a CTA adds its fp32 partial of each tile it touched to the split
+//   buffer with atomics.  While its first loads are in flight, each CTA also
+//   computes X A^T over its share of the 64-column blocks of K (fp32, CUDA
+//   cores) and adds it to the X A^T accumulator at its end.
+//   * Thread 0 streams the [256 rows x 128 bytes] code tile (128B-swizzled) and
+//     the four [m x 64] activation boxes of each step into a 3-deep ring (TMA).
+//   * 16 / kMT warps own 16 kMT weight rows each.  For every 64-column block
+//     they read their rows' code bytes, turn each byte into the two bf16 levels
+//     it encodes with one shared-memory load from a 256-entry pair table (one
+//     copy per lane: conflict-free), and feed them straight from registers to
+//     warp MMAs (m16n8k16, bf16 in, fp32 out): a code byte is exactly one
+//     A-fragment register.  The block's product is scaled by its constant
 //     c1' = fma(e4m3(q), c2/448, mu) and added to fp32 registers.
 //   * The tensor core here only replaces FMAs: per weight it does 2 M FLOP.
 //     Warp MMAs are used because a skinny-N product issued as tcgen05.mma
 //     from one thread costs about 80 cycles per 128x16x16 instruction, which
 //     caps a 16-token stream near 25 weights per cycle per SM, while HBM
 //     delivers about 46.
-//   * The last CTA to finish a tile (counter) adds s (X A^T) B^T and writes Y.
+//
+// k_finish: Y = bf16(split + s (X A^T) B^T), one thread per weight row.
+//
 // Numerics: the block constant multiplies the fp32 product of its block, so a
 // weight enters as bf16(L[code]) * c1' rather than bf16(L[code] * c1'): the same
 // linear map up to the rounding of each weight.
@@ -43,80 +48,140 @@ namespace qlora {
 namespace {
 
 constexpr int kRows = 256;                     // weight rows per tile
-constexpr int kComputeWarps = 16;              // 16 rows (one m16 MMA tile) each
-constexpr int kProducerWarp = kComputeWarps;
-constexpr int kThreads = (kComputeWarps + 1) * 32;
 constexpr int kStages = 3;
 constexpr int kStepCols = 256;                 // 4 blocks of 64 columns
-constexpr int kCodeTile = kRows * 128;         // 256 rows x 128 bytes, 128B-swizzled
-constexpr int kXBox = 16 * 128;                // 16 tokens x 64 bf16, 128B-swizzled
-constexpr int kXTile = 4 * kXBox;
-constexpr int kTable = 256 * 32 * 4;           // byte value x lane -> bf16 pair
-constexpr size_t kSmem = 32768 + kTable + kStages * (kCodeTile + kXTile) + 1024;
+constexpr uint32_t kCodeTile = kRows * 128;    // 256 rows x 128 bytes, 128B-swizzled
+constexpr uint32_t kXBox = 16 * 128;           // room for 16 tokens x 64 bf16, 128B-swizzled
+constexpr uint32_t kXTile = 4 * kXBox;
+// Shared-memory map (addresses in the CTA's shared window).  The pair table
+// sits at a 64 KB boundary so that one byte-permute builds a lookup address:
+// entry (code byte v, lane l) lives at kTableAddr + v * 256 + l * 4.  The other
+// half of each 256-byte row holds the block-constant slots.
+constexpr uint32_t kTableAddr = 0x10000;
+constexpr uint32_t kHighAddr = 0x20000;        // code stages 1 .. kStages - 1
+constexpr uint32_t kSmemTop = kHighAddr + (kStages - 1) * kCodeTile;
+constexpr uint32_t kMiscBytes = 256;           // barriers, levels
+constexpr size_t kSmemBytes = kSmemTop;        // enough for any start address of the window
 
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+// Predicated 16-byte load: when `pred` is false the registers are left as they
+// are (their contents are then unspecified and must not matter).
+__device__ __forceinline__ uint4 lds128_if(bool pred, uint32_t addr) {
   uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "@p ld.shared.v4.b32 {%0, %1, %2, %3}, [%5];\n\t}"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(static_cast<uint32_t>(pred)), "r"(addr));
   return v;
 }
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+// Pair-table read: the table does not change after set-up, so the load may be
+// scheduled freely (no volatile).
+__device__ __forceinline__ uint32_t lds_table(uint32_t addr) {
   uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
 }
-// Bounded barrier among the compute warps, built on an mbarrier (a named
-// bar.sync could not give up if a warp had left after a timed-out wait).
-__device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, uint32_t* err) {
-  mbar_arrive(bar);
-  const bool ok = mbar_wait(bar, phase, err);
-  phase ^= 1u;
-  return ok;
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
-// Byte t of the word, times 128, in bits 7..14 (rotate right by 8t - 7).
-__device__ __forceinline__ uint32_t byte_x128(uint32_t w, uint32_t rot) {
-  uint32_t r;
-  asm("shf.r.wrap.b32 %0, %1, %1, %2;" : "=r"(r) : "r"(w), "r"(rot));
-  return r & 0x7F80u;
+__device__ __forceinline__ void sts128(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+__device__ __forceinline__ float4 lds128f(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr) : "memory");
+  return v;
+}
+// Free half of pair-table row `row` (128 bytes at kTableAddr + row * 256 + 128).
+__device__ __forceinline__ uint32_t hole(uint32_t row, uint32_t byte) {
+  return kTableAddr + row * 256u + 128u + byte;
 }
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                                uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
       "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// Same with a zero accumulator input (the first product of a chain).
+__device__ __forceinline__ void mma_bf16_16816_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                                 uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
+// Four E4M3 bytes -> floats (exact: every E4M3 value is a normal f16 or zero).
+__device__ __forceinline__ void e4m3x4_to_f32(uint32_t q, float (&f)[4]) {
+  uint32_t lo, hi;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi) : "r"(q));
+  f[0] = __half2float(__ushort_as_half(static_cast<unsigned short>(lo & 0xFFFFu)));
+  f[1] = __half2float(__ushort_as_half(static_cast<unsigned short>(lo >> 16)));
+  f[2] = __half2float(__ushort_as_half(static_cast<unsigned short>(hi & 0xFFFFu)));
+  f[3] = __half2float(__ushort_as_half(static_cast<unsigned short>(hi >> 16)));
+}
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;");
 }
 
 // CTA i owns global steps [bound(i), bound(i + 1)) of all tiles, tile-major.
 __device__ __forceinline__ int64_t bound(int i, int64_t total, int ctas) {
   return (static_cast<int64_t>(i) * total) / ctas;
 }
-__device__ __forceinline__ int cta_of(int64_t x, int64_t total, int ctas) {
-  int i = static_cast<int>((x * ctas) / total);
-  while (i + 1 < ctas && bound(i + 1, total, ctas) <= x) ++i;
-  while (i > 0 && bound(i, total, ctas) > x) --i;
-  return i;
-}
 
-template <int kNT>   // n8 token tiles: 1 for M <= 8, 2 for M <= 16
-__global__ void __launch_bounds__(kThreads, 1)
+// Block-constant inputs of one step for one weight row, loaded ahead: the E4M3
+// bytes of the step's four blocks (byte b = block b) and c2 of the first
+// block's group (and, when K is not a multiple of 256 columns, of the last
+// block's group too).
+struct RowConsts {
+  uint32_t q;
+  float c2a, c2b;
+};
+
+// kMT m16 tiles (16 kMT weight rows) per warp, 16 / kMT warps per CTA.
+template <int kMT>
+struct GemvShape {
+  static constexpr int kWarps = 16 / kMT;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kRowsPerWarp = 16 * kMT;
+  static constexpr int kMaxRegs = kMT == 1 ? 112 : 224;
+};
+
+template <int kNT, bool kQuad, int kMT>   // kNT: n8 token tiles (1: M <= 8, 2: M <= 16); kQuad: K % 256 == 0
+__global__ void __maxnreg__(GemvShape<kMT>::kMaxRegs)
 k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
        const __grid_constant__ CUtensorMap xmap) {
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ float s_level[16];
-  __shared__ float s_xa[16 * 256];
-  __shared__ int s_last;
-
+  using S = GemvShape<kMT>;
+  constexpr int kWarps = S::kWarps;
+  constexpr int kThreads = S::kThreads;
+  constexpr int kRW = S::kRowsPerWarp;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw0 = smem_u32(smem_raw);
-  const uint32_t tbl = (raw0 + 32767u) & ~32767u;             // 32 KB aligned pair table
-  const uint32_t cs0 = tbl + kTable;                           // code tiles (1024-aligned)
-  const uint32_t xs0 = cs0 + kStages * kCodeTile;              // activation tiles
-  uint8_t* gen = smem_raw + (tbl - raw0);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(gen + kTable + kStages * (kCodeTile + kXTile));
+  uint32_t dyn_bytes;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_bytes));
+  const uint32_t xs0 = (raw0 + 1023u) & ~1023u;              // X stages (4 boxes each)
+  const uint32_t cs_low = xs0 + kStages * kXTile;            // code stage 0
+  const uint32_t misc = cs_low + kCodeTile;
+  if (misc + kMiscBytes > kTableAddr || raw0 + dyn_bytes < kSmemTop) {
+    if (threadIdx.x == 0) atomicOr(a.err, kErrSmemLayout);
+    return;
+  }
+  auto gptr = [&](uint32_t addr) { return smem_raw + (addr - raw0); };
+  auto code_stage = [&](uint32_t s) { return s == 0 ? cs_low : kHighAddr + (s - 1) * kCodeTile; };
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gptr(misc));
   uint64_t* full = bars;                  // codes + X landed (TMA)
-  uint64_t* empty = bars + kStages;       // one arrival per compute warp
-  uint64_t* gbar = bars + 2 * kStages;    // compute-warp barrier (all 256 threads)
+  uint64_t* empty = bars + kStages;       // one arrival per warp
+  float* s_level = reinterpret_cast<float*>(gptr(misc + 64));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -125,272 +190,423 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
   const int64_t x_beg = bound(blockIdx.x, total, gridDim.x);
   const int64_t x_end = bound(blockIdx.x + 1, total, gridDim.x);
   const int kblocks = static_cast<int>(a.kw / 64);
+  const int m = static_cast<int>(a.m);
 
-  if (threadIdx.x < 16) s_level[threadIdx.x] = a.level[threadIdx.x];
-  if (threadIdx.x == 0) {
+  // Position of a step: (tile, step within the tile's row of steps).  Advanced
+  // incrementally so that no 64-bit division runs per step.
+  struct Pos {
+    int tile, step;
+  };
+  auto advance = [&](Pos p) {
+    if (++p.step == steps) { p.step = 0; ++p.tile; }
+    return p;
+  };
+  const int64_t n_mine = x_end - x_beg;
+  const Pos first{static_cast<int>(x_beg / steps), static_cast<int>(x_beg % steps)};
+
+  // TMA issue (thread 0): iteration i goes to stage i % kStages once every warp
+  // has released that stage's previous iteration.
+  const uint32_t xbytes = 4u * static_cast<uint32_t>(m) * 128u;
+  const bool producer = threadIdx.x == 0;
+  Pos ppos = first;
+  int64_t pit = 0;
+  uint32_t ps = 0, pph = 0;
+  // issue the next step if its stage is free; `block` waits (bounded) for it
+  auto issue_next = [&](bool block) -> bool {
+    if (pit >= n_mine) return true;
+    if (!mbar_test_wait(&empty[ps], pph ^ 1u)) {
+      if (!block) return true;
+      if (!mbar_wait(&empty[ps], pph ^ 1u, a.err)) return false;
+    }
+    mbar_arrive_expect_tx(&full[ps], kCodeTile + xbytes);
+    const int col0 = ppos.step * kStepCols;
+    tma_load_2d(gptr(code_stage(ps)), &cmap, col0 / 2, ppos.tile * kRows, &full[ps]);
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+      tma_load_2d(gptr(xs0 + ps * kXTile + b * kXBox), &xmap, col0 + b * 64, 0, &full[ps]);
+    ppos = advance(ppos);
+    ++pit;
+    if (++ps == kStages) { ps = 0; pph ^= 1u; }
+    return true;
+  };
+  if (producer) {
+    // barriers first, then the first loads: they are in flight while the
+    // pair table is built
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kComputeWarps);
+      mbar_init(&empty[i], kWarps);
     }
-    mbar_init(gbar, kComputeWarps * 32);
     fence_barrier_init();
+    for (int i = 0; i < kStages - 1; ++i) issue_next(true);
   }
-  __syncthreads();
-  // pair table: entry (byte b, lane l) = {bf16(L[b >> 4]), bf16(L[b & 15])}, element order
-  for (int i = threadIdx.x; i < 256 * 32; i += kThreads) {
-    const int b = i >> 5, l = i & 31;
-    const __nv_bfloat162 v = __floats2bfloat162_rn(s_level[b >> 4], s_level[b & 15]);
-    asm volatile("st.shared.b32 [%0], %1;" ::"r"(tbl + b * 128 + l * 4),
-                 "r"(*reinterpret_cast<const uint32_t*>(&v)) : "memory");
-  }
-  __syncthreads();
 
-  if (warp == kProducerWarp) {
-    if (lane == 0) {
-      for (int64_t x = x_beg; x < x_end; ++x) {
-        const uint32_t it = static_cast<uint32_t>(x - x_beg);
-        const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
-        if (!mbar_wait(&empty[s], ph ^ 1u, a.err)) break;
-        const int tile = static_cast<int>(x / steps);
-        const int col0 = static_cast<int>(x % steps) * kStepCols;
-        mbar_arrive_expect_tx(&full[s], kCodeTile + kXTile);
-        tma_load_2d(gen + kTable + s * kCodeTile, &cmap, col0 / 2, tile * kRows, &full[s]);
+  // ------------------------------------------------ compute
+  // Lane (g, t) serves MMA rows g and g + 8 of the warp's kMT m16 tiles.  MMA
+  // row g of an 8-row group is weight row 8u + pg with pg = 2(g mod 4) + g / 4,
+  // so that the lanes of each half-warp read rows whose 128-byte swizzle
+  // patterns differ in bits 1 and 2 (no bank conflicts).  The lane's rows are
+  // warp*16kMT + 8q + pg (q < 2kMT; tile i uses q = 2i and 2i + 1).  In every
+  // 64-column block the lane reads the code bytes [8t, 8t + 8) of those rows.
+  // Columns enter the MMA in a permuted order (the same for X): slice j of a
+  // block feeds columns 16t + 4j + {0, 1} as k = {2t, 2t+1} and 16t + 4j + {2, 3}
+  // as k = {2t+8, 2t+9}, so every lane reads only its own bytes.
+  //
+  // Block constants: lane L computes the constants of weight row
+  // warp*16kMT + (L mod 16kMT) (all four blocks when kMT = 2, blocks
+  // 2(L / 16) and 2(L / 16) + 1 when kMT = 1) and stores them in a two-slot
+  // table in the free halves of pair-table rows 0..63; the lanes that read them
+  // belong to the same warp.
+  const int g = lane >> 2, t = lane & 3;
+  const int pg = ((g & 3) << 1) | (g >> 2);
+  const uint32_t tbase = kTableAddr | (static_cast<uint32_t>(lane) << 2);
+  const uint32_t crow = static_cast<uint32_t>(warp * kRW + pg) * 128u;
+  const float mu = __ldg(a.mean);
+  const uint32_t kbl = static_cast<uint32_t>(kblocks);
+
+  const int crow_l = warp * kRW + (lane & (kRW - 1));          // this lane's constant row
+  const int cb0 = kMT == 2 ? 0 : 2 * (lane >> 4);              // its first block
+  auto cblk0 = [&](Pos p) -> uint32_t {                        // block indices < 2^32
+    return static_cast<uint32_t>(p.tile * kRows + crow_l) * kbl + 4u * p.step;
+  };
+  auto load_raw = [&](Pos p, bool valid, RowConsts& k) {
+    k.q = 0;
+    k.c2a = 0.0f;
+    k.c2b = 0.0f;
+    if (valid && p.tile * kRows + crow_l < a.nw) {
+      const uint32_t blk0 = cblk0(p);
+      if (kQuad) {
+        k.q = __ldg(reinterpret_cast<const uint32_t*>(a.qabs + blk0));
+        k.c2a = __ldg(a.c2 + (blk0 >> 8));
+      } else {
+        const int nb = min(4, kblocks - 4 * p.step);
 #pragma unroll
         for (int b = 0; b < 4; ++b)
-          tma_load_2d(gen + kTable + kStages * kCodeTile + s * kXTile + b * kXBox, &xmap, col0 + b * 64, 0,
-                      &full[s]);
-      }
-    }
-    return;
-  }
-
-  // ------------------------------------------------ compute warps
-  const int g = lane >> 2, t = lane & 3;
-  const uint32_t tlane = tbl + lane * 4;
-  const uint32_t rot = (8u * t + 25u) & 31u;                   // 8t - 7 mod 32
-  const float mu = __ldg(a.mean);
-  float y[kNT][4];
-#pragma unroll
-  for (int n = 0; n < kNT; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) y[n][e] = 0.0f;
-
-  // Block-constant inputs (E4M3 byte, c2) of lane t's block in the warp's two
-  // rows, loaded two steps before their use (two register slots, alternating).
-  // qv[r] packs the E4M3 byte (bits 0..7) and the c2 group index (bits 8..);
-  // a row's group changes only every 256 blocks, so c2 / 448 is cached below.
-  auto load_raw = [&](int64_t xx, uint32_t (&qv)[2], float (&cv)[2]) {
-    const int tl = static_cast<int>(xx / steps);
-    const int kb = static_cast<int>(xx % steps) * 4 + t;
-    const int64_t r0 = static_cast<int64_t>(tl) * kRows + warp * 16 + g;
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int64_t n = r0 + 8 * r;
-      qv[r] = 0xFFFFFFFFu;                         // marks "no block": constant 0
-      cv[r] = 0.0f;
-      if (xx < x_end && n < a.nw && kb < kblocks) {
-        const int64_t blk = n * kblocks + kb;
-        qv[r] = __ldg(a.qabs + blk) | (static_cast<uint32_t>(blk >> 8) << 8);
-        cv[r] = __ldg(a.c2 + (blk >> 8));
+          if (b < nb) k.q |= static_cast<uint32_t>(__ldg(a.qabs + blk0 + b)) << (8 * b);
+        k.c2a = __ldg(a.c2 + (blk0 >> 8));
+        k.c2b = __ldg(a.c2 + ((blk0 + nb - 1) >> 8));
       }
     }
   };
-  uint32_t grp_cache[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
-  float c2q_cache[2] = {0.0f, 0.0f};
-
-  bool alive = true;
-  uint32_t gphase = 0;
-  // One step: wait for its stage, decode + multiply its four blocks, release
-  // the stage, and at the end of this CTA's share of a tile add the partial.
-  auto process = [&](int64_t x, uint32_t (&qv)[2], float (&cv)[2]) {
-    const uint32_t it = static_cast<uint32_t>(x - x_beg);
-    const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
-    const int tile = static_cast<int>(x / steps);
-    const int step = static_cast<int>(x % steps);
-    const int64_t row0 = static_cast<int64_t>(tile) * kRows + warp * 16 + g;   // rows row0, row0 + 8
-    float cmine[2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      cmine[r] = 0.0f;
-      if (qv[r] != 0xFFFFFFFFu) {
-        const uint32_t grp = qv[r] >> 8;
-        if (grp != grp_cache[r]) {
-          grp_cache[r] = grp;
-          c2q_cache[r] = __fdiv_rn(cv[r], 448.0f);
-        }
-        cmine[r] = block_constant(qv[r] & 0xFFu, c2q_cache[r], mu);
-      }
+  uint32_t grp_cache = 0xFFFFFFFFu;
+  float c2q_cache = 0.0f;
+  // c[b] = fma(e4m3(q_b), c2 / 448, mu) for the lane's row and blocks, into slot `slot`
+  auto write_consts = [&](Pos p, const RowConsts& k, uint32_t slot) {
+    const uint32_t blk0 = cblk0(p);
+    const uint32_t grp = blk0 >> 8;
+    if (grp != grp_cache) {
+      grp_cache = grp;
+      c2q_cache = __fdiv_rn(k.c2a, 448.0f);
     }
-    load_raw(x + 2, qv, cv);
-    if (!mbar_wait(&full[s], ph, a.err)) { alive = false; return; }
-    const uint32_t cs = cs0 + s * kCodeTile + (warp * 16 + g) * 128;
-    const uint32_t xs = xs0 + s * kXTile;
-#pragma unroll 2
-    for (int b = 0; b < 4; ++b) {
-      // code words of the two rows for block b (logical chunks 2b, 2b+1; swizzle key g)
-      uint32_t w[2][8];
+    float f[4];
+    e4m3x4_to_f32(k.q, f);
+    float c[4];
+    if (kQuad) {
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const uint32_t rb = cs + r * 8 * 128;
-        const uint4 lo = lds128(rb + (((2 * b) ^ g) << 4));
-        const uint4 hi = lds128(rb + (((2 * b + 1) ^ g) << 4));
-        w[r][0] = lo.x; w[r][1] = lo.y; w[r][2] = lo.z; w[r][3] = lo.w;
-        w[r][4] = hi.x; w[r][5] = hi.y; w[r][6] = hi.z; w[r][7] = hi.w;
-      }
-      float p[2][kNT][4];                           // two chains: even / odd slices
+      for (int b = 0; b < 4; ++b) c[b] = __fmaf_rn(f[b], c2q_cache, mu);
+    } else {
+      const float c2q_b = __fdiv_rn(k.c2b, 448.0f);
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
-#pragma unroll
-        for (int n = 0; n < kNT; ++n)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) p[c][n][e] = 0.0f;
-      const uint32_t xb = xs + b * kXBox;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {               // 16-column slices of the block
-        uint32_t bf[kNT][2];
-#pragma unroll
-        for (int n = 0; n < kNT; ++n) {
-          const uint32_t xr = xb + (8 * n + g) * 128 + 4 * t;
-          bf[n][0] = lds32(xr + (((2 * j) ^ g) << 4));
-          bf[n][1] = lds32(xr + (((2 * j + 1) ^ g) << 4));
-        }
-        const uint32_t a0 = lds32(tlane | byte_x128(w[0][2 * j], rot));
-        const uint32_t a1 = lds32(tlane | byte_x128(w[1][2 * j], rot));
-        const uint32_t a2 = lds32(tlane | byte_x128(w[0][2 * j + 1], rot));
-        const uint32_t a3 = lds32(tlane | byte_x128(w[1][2 * j + 1], rot));
-#pragma unroll
-        for (int n = 0; n < kNT; ++n) mma_bf16_16816(p[j & 1][n], a0, a1, a2, a3, bf[n][0], bf[n][1]);
-      }
-      // scale the block's partial by its constants (rows g and g+8)
-      const float c_lo = __shfl_sync(0xFFFFFFFFu, cmine[0], (lane & ~3) | b);
-      const float c_hi = __shfl_sync(0xFFFFFFFFu, cmine[1], (lane & ~3) | b);
-#pragma unroll
-      for (int n = 0; n < kNT; ++n) {
-        y[n][0] = __fmaf_rn(c_lo, p[0][n][0] + p[1][n][0], y[n][0]);
-        y[n][1] = __fmaf_rn(c_lo, p[0][n][1] + p[1][n][1], y[n][1]);
-        y[n][2] = __fmaf_rn(c_hi, p[0][n][2] + p[1][n][2], y[n][2]);
-        y[n][3] = __fmaf_rn(c_hi, p[0][n][3] + p[1][n][3], y[n][3]);
-      }
+      for (int b = 0; b < 4; ++b) c[b] = __fmaf_rn(f[b], ((blk0 + b) >> 8) == grp ? c2q_cache : c2q_b, mu);
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
+    const uint32_t e = slot * 256u + static_cast<uint32_t>(crow_l);
+    if (kMT == 2) {
+      sts128(hole(e >> 3, (e & 7u) * 16u), c[0], c[1], c[2], c[3]);
+    } else {
+      const float c0 = cb0 == 0 ? c[0] : c[2], c1 = cb0 == 0 ? c[1] : c[3];
+      asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(hole(e >> 3, (e & 7u) * 16u + cb0 * 4u)),
+                   "f"(c0), "f"(c1) : "memory");
+    }
+  };
 
-    if (step == steps - 1 || x == x_end - 1) {
-      // end of this CTA's share of the tile: add the partial, maybe finish the tile
+  Pos pos = first;
+  Pos pos1 = advance(pos), pos2 = advance(pos1), pos3 = advance(pos2);
+  RowConsts r0, ra, rb;                   // raw inputs of steps 0, it + 1 and it + 2
+  load_raw(pos, n_mine > 0, r0);
+  load_raw(pos1, n_mine > 1, ra);
+  load_raw(pos2, n_mine > 2, rb);
+
+  if (threadIdx.x < 16) s_level[threadIdx.x] = a.level[threadIdx.x];
+  __syncthreads();                        // levels, barrier initialisation
+  // pair table: entry (byte v, lane l) = {bf16(L[v >> 4]), bf16(L[v & 15])}, element order
+  for (int i = threadIdx.x; i < 256 * 32; i += kThreads) {
+    const int v = i >> 5, l = i & 31;
+    const __nv_bfloat162 e = __floats2bfloat162_rn(s_level[v >> 4], s_level[v & 15]);
+    sts32(kTableAddr + v * 256 + l * 4, *reinterpret_cast<const uint32_t*>(&e));
+  }
+  write_consts(pos, r0, 0);
+  // X A^T over this CTA's 64-column blocks of K (blocks blockIdx.x + i * gridDim.x),
+  // while the first code tiles are in flight.  The block's A slice [r x 64]
+  // goes to code stage 2 (not loaded before the main loop; chunk c of row j at
+  // ((c + j) mod 8) so that a quarter-warp reading chunk c of eight rows hits
+  // distinct banks), its X slice [m x 64] to pair-table holes 64..79, and the
+  // fp32 partial (m x r) stays in holes 128..255 until the end of the kernel.
+  const int xa_n = m * a.r;                // <= 16 * 256 floats
+  auto xa_hole = [](int e) { return hole(128u + (e >> 5), (e & 31) * 4u); };
+  const uint32_t a_stage = code_stage(2);
+  for (int kb = blockIdx.x; kb < kblocks; kb += gridDim.x) {
+    __syncthreads();                      // previous block's slices consumed
+    for (int e = threadIdx.x; e < a.r * 8; e += kThreads) {
+      const int j = e >> 3, ch = e & 7;
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.lora_a + static_cast<int64_t>(j) * a.kw + kb * 64) + ch);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_stage + j * 128u + ((ch + j) & 7) * 16u),
+                   "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+    }
+    for (int e = threadIdx.x; e < m * 8; e += kThreads) {
+      const int i = e >> 3, ch = e & 7;
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<int64_t>(i) * a.kw + kb * 64) + ch);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(hole(64u + i, ch * 16u)),
+                   "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < xa_n; e += kThreads) {
+      const int i = e / a.r, j = e % a.r;
+      float acc = kb == static_cast<int>(blockIdx.x) ? 0.0f : __uint_as_float(lds_table(xa_hole(e)));
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        uint4 av, xv;
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(av.x), "=r"(av.y), "=r"(av.z), "=r"(av.w)
+                     : "r"(a_stage + j * 128u + ((ch + j) & 7) * 16u));
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(xv.x), "=r"(xv.y), "=r"(xv.z), "=r"(xv.w)
+                     : "r"(hole(64u + i, ch * 16u)));
+        acc = __fmaf_rn(bf16_lo(av.x), bf16_lo(xv.x), acc);
+        acc = __fmaf_rn(bf16_hi(av.x), bf16_hi(xv.x), acc);
+        acc = __fmaf_rn(bf16_lo(av.y), bf16_lo(xv.y), acc);
+        acc = __fmaf_rn(bf16_hi(av.y), bf16_hi(xv.y), acc);
+        acc = __fmaf_rn(bf16_lo(av.z), bf16_lo(xv.z), acc);
+        acc = __fmaf_rn(bf16_hi(av.z), bf16_hi(xv.z), acc);
+        acc = __fmaf_rn(bf16_lo(av.w), bf16_lo(xv.w), acc);
+        acc = __fmaf_rn(bf16_hi(av.w), bf16_hi(xv.w), acc);
+      }
+      sts32(xa_hole(e), __float_as_uint(acc));
+    }
+  }
+  fence_proxy_async_smem();               // stage 2 is written by TMA from here on
+  __syncthreads();                        // pair table, step 0's constants, X A^T partial in place
+  launch_dependents();                    // k_finish may be scheduled; it waits for this grid
+
+  // X rows of this lane (token 8n + g); lanes of tokens >= m load nothing, and
+  // the MMA columns they feed are never stored.
+  bool xon[kNT];
+  uint32_t xoff[kNT][2];
+#pragma unroll
+  for (int n = 0; n < kNT; ++n) {
+    xon[n] = 8 * n + g < m;
+#pragma unroll
+    for (int jp = 0; jp < 2; ++jp) xoff[n][jp] = (8 * n + g) * 128 + ((((2u * t) + jp) ^ g) << 4);
+  }
+
+  float y[kMT][kNT][4];
+#pragma unroll
+  for (int i = 0; i < kMT; ++i)
+#pragma unroll
+    for (int n = 0; n < kNT; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) y[i][n][e] = 0.0f;
+  // The partial of the first tile this CTA touches is kept in registers until
+  // the next tile boundary (or the end of the range): by then the previous
+  // kernel (zeroing of the accumulators) has surely finished, so the wait for
+  // it does not stall the stream.
+  float ys[kMT][kNT][4];
+  int ys_tile = -1;
+  bool dep_done = false;
+  // add a tile partial to the split buffer (fire-and-forget reductions)
+  auto flush = [&](int tile, float (&v)[kMT][kNT][4]) {
+#pragma unroll
+    for (int i = 0; i < kMT; ++i)
 #pragma unroll
       for (int n = 0; n < kNT; ++n)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int64_t row = row0 + 8 * (e >> 1);
+          const int64_t row = static_cast<int64_t>(tile) * kRows + warp * kRW + 8 * (2 * i + (e >> 1)) + pg;
           const int tok = 8 * n + 2 * t + (e & 1);
-          if (row < a.nw && tok < a.m) atomicAdd(a.yacc + tok * a.nw + row, y[n][e]);
-          y[n][e] = 0.0f;
+          if (row < a.nw && tok < m) atomicAdd(a.yacc + tok * a.nw + row, v[i][n][e]);
         }
-      __threadfence();
-      if (!group_sync(gbar, gphase, a.err)) { alive = false; return; }
-      if (threadIdx.x == 0) {
-        const int first = cta_of(static_cast<int64_t>(tile) * steps, total, gridDim.x);
-        const int last = cta_of(static_cast<int64_t>(tile + 1) * steps - 1, total, gridDim.x);
-        s_last = (atomicAdd(a.counters + tile, 1) == last - first) ? 1 : 0;
-      }
-      if (!group_sync(gbar, gphase, a.err)) { alive = false; return; }
-      if (s_last) {
-        __threadfence();
-        for (int e = threadIdx.x; e < a.m * a.r; e += kComputeWarps * 32)
-          s_xa[e] = __ldcg(a.xa + (e / a.r) * a.ld_xa + (e % a.r));
-        if (!group_sync(gbar, gphase, a.err)) { alive = false; return; }
-        const int64_t n = static_cast<int64_t>(tile) * kRows + threadIdx.x;
-        if (threadIdx.x < kRows && n < a.nw) {
-          float lo[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) lo[i] = 0.0f;
-          const uint4* brow = reinterpret_cast<const uint4*>(a.lora_b + n * a.r);
-          for (int c = 0; c < a.r / 8; ++c) {
-            const uint4 bv = __ldg(brow + c);
-            const float b8[8] = {bf16_lo(bv.x), bf16_hi(bv.x), bf16_lo(bv.y), bf16_hi(bv.y),
-                                 bf16_lo(bv.z), bf16_hi(bv.z), bf16_lo(bv.w), bf16_hi(bv.w)};
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              if (i < a.m) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) lo[i] = __fmaf_rn(s_xa[i * a.r + c * 8 + e], b8[e], lo[i]);
-              }
-          }
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            if (i < a.m) {
-              const float acc = __ldcg(a.yacc + i * a.nw + n);
-              const __nv_bfloat16 v = __float2bfloat16_rn(__fmaf_rn(a.s, lo[i], acc));
-              a.y[i * a.nw + n] = *reinterpret_cast<const uint16_t*>(&v);
-            }
-          }
-        }
-        if (!group_sync(gbar, gphase, a.err)) { alive = false; return; }
-      }
-    }
   };
 
-  uint32_t qa[2], qb[2];
-  float ca[2], cb[2];
-  load_raw(x_beg, qa, ca);
-  load_raw(x_beg + 1, qb, cb);
-  for (int64_t x = x_beg; x < x_end && alive; x += 2) {
-    process(x, qa, ca);
-    if (x + 1 < x_end && alive) process(x + 1, qb, cb);
+  uint32_t s = 0, ph = 0;
+  bool alive = true;
+  for (int64_t it = 0; it < n_mine && alive; ++it) {
+    // this step's constants c[q][b] for the lane's rows warp*16kMT + 8q + pg
+    float c[2 * kMT][4];
+    const uint32_t cslot = static_cast<uint32_t>(it & 1) * 256u;
+#pragma unroll
+    for (int q = 0; q < 2 * kMT; ++q) {
+      const uint32_t e = cslot + static_cast<uint32_t>(warp * kRW + 8 * q + pg);
+      const float4 v = lds128f(hole(e >> 3, (e & 7u) * 16u));
+      c[q][0] = v.x; c[q][1] = v.y; c[q][2] = v.z; c[q][3] = v.w;
+    }
+    // the stage of this step: test first (cheap when the data is already there)
+    if (!mbar_test_wait(&full[s], ph) && !mbar_wait(&full[s], ph, a.err)) break;
+    const uint32_t cs = code_stage(s) + crow;
+    const uint32_t xs = xs0 + s * kXTile;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const uint32_t coff = ((((2u * b) + (t >> 1)) ^ pg) << 4) | ((t & 1u) << 3);
+      uint2 cw[2 * kMT];
+#pragma unroll
+      for (int q = 0; q < 2 * kMT; ++q) cw[q] = lds64(cs + q * 1024u + coff);
+      uint4 xv[kNT][2];
+#pragma unroll
+      for (int n = 0; n < kNT; ++n)
+#pragma unroll
+        for (int jp = 0; jp < 2; ++jp) xv[n][jp] = lds128_if(xon[n], xs + b * kXBox + xoff[n][jp]);
+      if (b == 3) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);                // stage fully read
+      }
+      if (b == 1) {
+        // next step's constants into the other slot (read two steps ago by
+        // this warp; the syncwarp at b == 3 orders them before their readers)
+        __syncwarp();
+        if (it + 1 < n_mine) write_consts(pos1, ra, static_cast<uint32_t>((it + 1) & 1));
+      }
+      if (producer && !issue_next(b == 3)) { alive = false; break; }
+      float p[kMT][kNT][4];                                   // [m tile][n tile][element]
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t sel0 = 0x7604u | ((2u * (j & 1)) << 4);   // byte 2(j&1) of the word
+        const uint32_t sel1 = sel0 + 0x10u;                      // byte 2(j&1) + 1
+#pragma unroll
+        for (int i = 0; i < kMT; ++i) {
+          const uint32_t w0 = (j < 2) ? cw[2 * i].x : cw[2 * i].y;
+          const uint32_t w1 = (j < 2) ? cw[2 * i + 1].x : cw[2 * i + 1].y;
+          const uint32_t a0 = lds_table(__byte_perm(w0, tbase, sel0));
+          const uint32_t a1 = lds_table(__byte_perm(w1, tbase, sel0));
+          const uint32_t a2 = lds_table(__byte_perm(w0, tbase, sel1));
+          const uint32_t a3 = lds_table(__byte_perm(w1, tbase, sel1));
+#pragma unroll
+          for (int n = 0; n < kNT; ++n) {
+            const uint32_t b0 = (j & 1) ? xv[n][j >> 1].z : xv[n][j >> 1].x;
+            const uint32_t b1 = (j & 1) ? xv[n][j >> 1].w : xv[n][j >> 1].y;
+            if (j == 0) mma_bf16_16816_z(p[i][n], a0, a1, a2, a3, b0, b1);
+            else mma_bf16_16816(p[i][n], a0, a1, a2, a3, b0, b1);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kMT; ++i)
+#pragma unroll
+        for (int n = 0; n < kNT; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) y[i][n][e] = __fmaf_rn(c[2 * i + (e >> 1)][b], p[i][n][e], y[i][n][e]);
+    }
+    if (!alive) break;
+
+    if (pos.step == steps - 1 || it == n_mine - 1) {
+      // end of this CTA's share of the tile
+      if (!dep_done && ys_tile < 0 && it != n_mine - 1) {
+        ys_tile = pos.tile;                                   // keep it for later
+#pragma unroll
+        for (int i = 0; i < kMT; ++i)
+#pragma unroll
+          for (int n = 0; n < kNT; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) ys[i][n][e] = y[i][n][e];
+      } else {
+        if (!dep_done) {
+          grid_dependency_wait();
+          dep_done = true;
+        }
+        if (ys_tile >= 0) {
+          flush(ys_tile, ys);
+          ys_tile = -1;
+        }
+        flush(pos.tile, y);
+      }
+#pragma unroll
+      for (int i = 0; i < kMT; ++i)
+#pragma unroll
+        for (int n = 0; n < kNT; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) y[i][n][e] = 0.0f;
+    }
+    ra = rb;                                   // loaded a full step ago
+    load_raw(pos3, it + 3 < n_mine, rb);
+    pos = pos1; pos1 = pos2; pos2 = pos3; pos3 = advance(pos3);
+    if (++s == kStages) { s = 0; ph ^= 1u; }
+  }
+  if (!alive) return;
+  if (blockIdx.x < kblocks) {
+    if (!dep_done) grid_dependency_wait();
+    for (int e = threadIdx.x; e < xa_n; e += kThreads)
+      atomicAdd(a.xa + (e / a.r) * a.ld_xa + (e % a.r), __uint_as_float(lds_table(xa_hole(e))));
   }
 }
 
-// X A^T for M <= 16 tokens: block j reduces column j over all of K in fp32.
-// Also zeroes k_gemv's split buffer and tile counters (grid-stride).
-__global__ void __launch_bounds__(256)
-k_xa_small(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A, int64_t m, int64_t kw, int r,
-           float* __restrict__ xa, int64_t ld, float* __restrict__ xa_out, float* __restrict__ zero_f,
-           int64_t zero_n, int* __restrict__ zero_i, int zero_ni) {
-  __shared__ float s_red[8][16];
-  const int j = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float acc[16];
+// Zeroes the accumulators of k_gemv.  k_gemv is launched as its programmatic
+// dependent: it starts streaming the weight at once and waits for this grid
+// only before its first atomic.
+__global__ void __launch_bounds__(256) k_gemv_zero(float4* __restrict__ a, int64_t n4a, float4* __restrict__ b,
+                                                   int64_t n4b) {
+  launch_dependents();
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const float4 z = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  for (int64_t i = gtid; i < n4a; i += nthreads) a[i] = z;
+  for (int64_t i = gtid; i < n4b; i += nthreads) b[i] = z;
+}
+
+// Y[i, n] = bf16(split[i, n] + s * sum_c XA[i, c] B[n, c]), one thread per row n.
+__global__ void __launch_bounds__(128)
+k_finish(const float* __restrict__ yacc, const float* __restrict__ xa, int64_t ld_xa,
+         const uint16_t* __restrict__ lora_b, int r, float s, int64_t m, int64_t nw, uint16_t* __restrict__ y,
+         float* __restrict__ xa_out) {
+  __shared__ float s_xa[16 * 256];
+  grid_dependency_wait();                  // k_gemv complete (it waited for k_gemv_zero)
+  for (int e = threadIdx.x; e < m * r; e += blockDim.x) {
+    const float v = __ldcg(xa + (e / r) * ld_xa + (e % r));
+    s_xa[e] = v;
+    if (xa_out && blockIdx.x == 0) xa_out[e] = v;
+  }
+  __syncthreads();
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (n >= nw) return;
+  float lo[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
-  const int64_t nchunks = kw / 8;
-  for (int64_t c = threadIdx.x; c < nchunks; c += blockDim.x) {
-    const uint4 av = __ldg(reinterpret_cast<const uint4*>(A + j * kw) + c);
-    const float af[8] = {bf16_lo(av.x), bf16_hi(av.x), bf16_lo(av.y), bf16_hi(av.y),
-                         bf16_lo(av.z), bf16_hi(av.z), bf16_lo(av.w), bf16_hi(av.w)};
+  for (int i = 0; i < 16; ++i) lo[i] = 0.0f;
+  const uint4* brow = reinterpret_cast<const uint4*>(lora_b + n * r);
+  for (int c0 = 0; c0 < r / 8; c0 += 8) {            // eight 16-byte loads in flight at a time
+    uint4 bv[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if (i < m) {
-        const uint4 xv = __ldg(reinterpret_cast<const uint4*>(X + i * kw) + c);
-        const float xf[8] = {bf16_lo(xv.x), bf16_hi(xv.x), bf16_lo(xv.y), bf16_hi(xv.y),
-                             bf16_lo(xv.z), bf16_hi(xv.z), bf16_lo(xv.w), bf16_hi(xv.w)};
+    for (int u = 0; u < 8; ++u) bv[u] = (c0 + u < r / 8) ? __ldg(brow + c0 + u) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[i] = __fmaf_rn(af[e], xf[e], acc[i]);
-      }
+    for (int u = 0; u < 8; ++u) {
+      if (c0 + u >= r / 8) break;
+      const int cc = c0 + u;
+      const float b8[8] = {bf16_lo(bv[u].x), bf16_hi(bv[u].x), bf16_lo(bv[u].y), bf16_hi(bv[u].y),
+                           bf16_lo(bv[u].z), bf16_hi(bv[u].z), bf16_lo(bv[u].w), bf16_hi(bv[u].w)};
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (i < m) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) lo[i] = __fmaf_rn(s_xa[i * r + cc * 8 + e], b8[e], lo[i]);
+        }
     }
   }
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc[i] += __shfl_xor_sync(0xFFFFFFFFu, acc[i], o);
+    if (i < m) {
+      const __nv_bfloat16 v = __float2bfloat16_rn(__fmaf_rn(s, lo[i], __ldcg(yacc + i * nw + n)));
+      y[i * nw + n] = *reinterpret_cast<const uint16_t*>(&v);
+    }
   }
-  if (lane == 0) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) s_red[warp][i] = acc[i];
-  }
-  __syncthreads();
-  if (threadIdx.x < m) {
-    float v = 0.0f;
-    for (int w = 0; w < 8; ++w) v += s_red[w][threadIdx.x];
-    xa[threadIdx.x * ld + j] = v;
-    if (xa_out) xa_out[threadIdx.x * r + j] = v;
-  }
-  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  for (int64_t i = gtid; i < zero_n; i += nthreads) zero_f[i] = 0.0f;
-  for (int64_t i = gtid; i < zero_ni; i += nthreads) zero_i[i] = 0;
 }
 
-template <int kNT>
+cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, void** args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+template <int kNT, bool kQuad, int kMT>
 cudaError_t launch_gemv_t(const GemvArgs& args, const CUtensorMap& cm, const CUtensorMap& xm, int num_sms,
                           cudaStream_t stream) {
   static std::atomic<uint64_t> attr_done{0};
@@ -399,31 +615,59 @@ cudaError_t launch_gemv_t(const GemvArgs& args, const CUtensorMap& cm, const CUt
   if (e != cudaSuccess) return e;
   const uint64_t bit = 1ull << (dev & 63);
   if (!(attr_done.load(std::memory_order_acquire) & bit)) {
-    e = cudaFuncSetAttribute(k_gemv<kNT>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
+    e = cudaFuncSetAttribute(k_gemv<kNT, kQuad, kMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes));
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(bit, std::memory_order_acq_rel);
   }
   const int64_t total = static_cast<int64_t>(args.m_tiles) * args.steps;
-  const int grid = static_cast<int>(total < num_sms ? total : num_sms);
-  k_gemv<kNT><<<grid, kThreads, kSmem, stream>>>(args, cm, xm);
-  return cudaGetLastError();
+  const unsigned grid = static_cast<unsigned>(total < num_sms ? total : num_sms);
+  GemvArgs a = args;
+  CUtensorMap c = cm, x = xm;
+  void* kargs[3] = {&a, &c, &x};
+  return launch_pdl(reinterpret_cast<const void*>(k_gemv<kNT, kQuad, kMT>), dim3(grid),
+                    dim3(GemvShape<kMT>::kThreads), kSmemBytes, stream, kargs);
+}
+
+template <int kMT>
+cudaError_t launch_gemv_mt(const GemvArgs& args, const CUtensorMap& cm, const CUtensorMap& xm, int num_sms,
+                           cudaStream_t stream) {
+  const bool quad = (args.kw / 64) % 4 == 0;
+  if (args.m <= 8)
+    return quad ? launch_gemv_t<1, true, kMT>(args, cm, xm, num_sms, stream)
+                : launch_gemv_t<1, false, kMT>(args, cm, xm, num_sms, stream);
+  return quad ? launch_gemv_t<2, true, kMT>(args, cm, xm, num_sms, stream)
+              : launch_gemv_t<2, false, kMT>(args, cm, xm, num_sms, stream);
 }
 
 }  // namespace
 
 int gemv_tile_rows() { return kRows; }
 
-cudaError_t launch_xa_small(const uint16_t* X, const uint16_t* A, int64_t m, int64_t kw, int r, float* xa,
-                            int64_t ld, float* xa_out, float* zero_f, int64_t zero_n, int* zero_i,
-                            int zero_ni, cudaStream_t stream) {
-  k_xa_small<<<r, 256, 0, stream>>>(X, A, m, kw, r, xa, ld, xa_out, zero_f, zero_n, zero_i, zero_ni);
+cudaError_t launch_gemv_zero(float* a, int64_t n_a, float* b, int64_t n_b, cudaStream_t stream) {
+  const int64_t n4 = (n_a > n_b ? n_a : n_b) / 4;
+  int64_t grid = (n4 + 255) / 256;
+  if (grid > 1024) grid = 1024;
+  if (grid < 1) grid = 1;
+  k_gemv_zero<<<static_cast<unsigned>(grid), 256, 0, stream>>>(reinterpret_cast<float4*>(a), n_a / 4,
+                                                               reinterpret_cast<float4*>(b), n_b / 4);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemv(const GemvArgs& args, const CUtensorMap& codes_map, const CUtensorMap& x_map,
                         int num_sms, cudaStream_t stream) {
-  if (args.m <= 8) return launch_gemv_t<1>(args, codes_map, x_map, num_sms, stream);
-  return launch_gemv_t<2>(args, codes_map, x_map, num_sms, stream);
+#ifdef GEMV_FORCE_MT
+  return launch_gemv_mt<GEMV_FORCE_MT>(args, codes_map, x_map, num_sms, stream);
+#else
+  return launch_gemv_mt<2>(args, codes_map, x_map, num_sms, stream);
+#endif
+}
+
+cudaError_t launch_gemv_finish(const float* yacc, const float* xa, int64_t ld_xa, const uint16_t* lora_b, int r,
+                               float s, int64_t m, int64_t nw, uint16_t* y, float* xa_out, cudaStream_t stream) {
+  void* kargs[10] = {&yacc, &xa, &ld_xa, &lora_b, &r, &s, &m, &nw, &y, &xa_out};
+  const unsigned grid = static_cast<unsigned>((nw + 127) / 128);
+  return launch_pdl(reinterpret_cast<const void*>(k_finish), dim3(grid), dim3(128), 0, stream, kargs);
 }
 
 }  // namespace qlora

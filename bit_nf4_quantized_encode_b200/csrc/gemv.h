@@ -13,14 +13,12 @@ struct GemvArgs {
   const float* mean;         // per-tensor mean
   int64_t nw, kw;            // W shape (rows = out features, cols = in features)
   int64_t m;                 // token rows (<= 16)
-  float* yacc;               // fp32 [m, nw] accumulator, zero on entry
-  int* counters;             // [m_tiles] finished shares per tile, zero on entry
-  const float* xa;           // X A^T, fp32 [m, ld_xa]
+  float* yacc;               // fp32 [m, nw] accumulator, zeroed by k_gemv_zero
+  const uint16_t* x;         // X bf16 [m, kw]
+  const uint16_t* lora_a;    // LoRA A bf16 [r, kw]
+  float* xa;                 // fp32 [m, ld_xa] accumulator of X A^T, zeroed by k_gemv_zero
   int64_t ld_xa;
-  const uint16_t* lora_b;    // LoRA B [nw, r] bf16
   int r;
-  float s;                   // LoRA scale
-  uint16_t* y;               // bf16 [m, nw] output
   int m_tiles;               // tiles of gemv_tile_rows() weight rows
   int steps;                 // 256-column steps per row
   float level[16];           // NF4 levels
@@ -29,15 +27,19 @@ struct GemvArgs {
 
 int gemv_tile_rows();
 
-// X A^T (fp32 [m, ld] and optionally [m, r] copy) for m <= 16 tokens, plus
-// zeroing of zero_f[zero_n] and zero_i[zero_ni] for k_gemv.
-cudaError_t launch_xa_small(const uint16_t* X, const uint16_t* A, int64_t m, int64_t kw, int r, float* xa,
-                            int64_t ld, float* xa_out, float* zero_f, int64_t zero_n, int* zero_i,
-                            int zero_ni, cudaStream_t stream);
+// Zeroes the two fp32 accumulators of k_gemv (n_a and n_b floats, multiples of 4).
+cudaError_t launch_gemv_zero(float* a, int64_t n_a, float* b, int64_t n_b, cudaStream_t stream);
 
 // codes_map: packed codes as uint8 [nw, kw/2], box {128, 256}, 128-byte swizzle.
-// x_map: X bf16 [m, kw], box {64, 16}, 128-byte swizzle.
+// x_map: X bf16 [m, kw], box {64, m}, 128-byte swizzle.
+// k_gemv is launched as a programmatic dependent of the kernel before it in the
+// stream, which must be k_gemv_zero of the same call.
 cudaError_t launch_gemv(const GemvArgs& args, const CUtensorMap& codes_map, const CUtensorMap& x_map,
                         int num_sms, cudaStream_t stream);
+
+// Y = bf16(yacc + s (X A^T) B^T), and X A^T into xa_out [m, r] when not null;
+// launched as the programmatic dependent of k_gemv.
+cudaError_t launch_gemv_finish(const float* yacc, const float* xa, int64_t ld_xa, const uint16_t* lora_b, int r,
+                               float s, int64_t m, int64_t nw, uint16_t* y, float* xa_out, cudaStream_t stream);
 
 }  // namespace qlora

@@ -83,6 +83,7 @@ Nf4Tables build() {
   // For each bucket find the float interval [lo, hi] of n in [-1, 1] that the
   // kernel's bucket formula maps to it (monotone, so bisect on float order).
   t.ok = true;
+  t.fast_ok = true;
   const uint32_t kmin = ordered_key(-1.0f), kmax = ordered_key(1.0f);
   for (int u = 0; u < kNumBuckets; ++u) {
     uint32_t lo = kmin, hi = kmax;  // first key with bucket >= u
@@ -110,6 +111,11 @@ Nf4Tables build() {
       else if (t.threshold[i] <= nhi) { ++inside; thr = t.threshold[i]; }
     }
     if (inside > 1) t.ok = false;
+    // The encoder's reciprocal path only re-checks the threshold of the bucket
+    // its estimate falls in; that is exact when no threshold is within 2^-20
+    // of a bucket edge (the estimate is within 2^-22 of the IEEE quotient).
+    if (inside == 1 && (static_cast<double>(thr) - nlo <= 0x1.0p-20 || nhi - static_cast<double>(thr) <= 0x1.0p-20))
+      t.fast_ok = false;
     t.bucket_base[u] = static_cast<uint8_t>(base);
     t.bucket_thr[u] = thr;
   }

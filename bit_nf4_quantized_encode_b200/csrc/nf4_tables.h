@@ -15,6 +15,7 @@ struct Nf4Tables {
   float bucket_thr[kNumBuckets];     // the one threshold inside bucket u, or +inf
   uint8_t bucket_base[kNumBuckets];  // code of the smallest n in bucket u
   bool ok;                    // every bucket holds at most one threshold
+  bool fast_ok;               // every threshold lies more than 2^-20 inside its bucket
 };
 
 // Built once (thread-safe) on first use.

@@ -96,6 +96,8 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const uint16_t* W, const q
     et.bucket_thr[i] = i < kNumBuckets ? tabs.bucket_thr[i] : INFINITY;
     et.bucket_base[i] = i < kNumBuckets ? tabs.bucket_base[i] : 15;
   }
+  et.fast = tabs.fast_ok ? 1 : 0;
+
   const int64_t nblocks = (numel + 63) / 64;
   float* c1buf = static_cast<float*>(scratch);
   double* partials = reinterpret_cast<double*>(static_cast<unsigned char*>(scratch) + kNoAllocC1Bytes);

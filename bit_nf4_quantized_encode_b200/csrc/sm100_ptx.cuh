@@ -15,6 +15,7 @@ namespace qlora {
 enum : uint32_t {
   kErrWaitTimeout = 1u << 0,   // an mbarrier wait gave up
   kErrTmemAlloc   = 1u << 1,   // TMEM allocation returned an unexpected address
+  kErrSmemLayout  = 1u << 2,   // the shared-memory window does not fit a kernel's fixed map
 };
 
 // Bound on any single mbarrier wait, in SM clock cycles (about two seconds at
@@ -58,6 +59,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+// Non-blocking check of a phase (returns at once).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
   return ok != 0;
