@@ -48,20 +48,26 @@ namespace qlora {
 namespace {
 
 constexpr int kRows = 256;                     // weight rows per tile
-constexpr int kStages = 3;
 constexpr int kStepCols = 256;                 // 4 blocks of 64 columns
 constexpr uint32_t kCodeTile = kRows * 128;    // 256 rows x 128 bytes, 128B-swizzled
-constexpr uint32_t kXBox = 16 * 128;           // room for 16 tokens x 64 bf16, 128B-swizzled
-constexpr uint32_t kXTile = 4 * kXBox;
 // Shared-memory map (addresses in the CTA's shared window).  The pair table
 // sits at a 64 KB boundary so that one byte-permute builds a lookup address:
 // entry (code byte v, lane l) lives at kTableAddr + v * 256 + l * 4.  The other
-// half of each 256-byte row holds the block-constant slots.
+// half of each 256-byte row holds the block-constant slots, X A^T staging and
+// partial.  Below the table: the X stages and code stage 0; above it: code
+// stages 1 .. kStages - 1.
 constexpr uint32_t kTableAddr = 0x10000;
-constexpr uint32_t kHighAddr = 0x20000;        // code stages 1 .. kStages - 1
-constexpr uint32_t kSmemTop = kHighAddr + (kStages - 1) * kCodeTile;
+constexpr uint32_t kHighAddr = 0x20000;
 constexpr uint32_t kMiscBytes = 256;           // barriers, levels
-constexpr size_t kSmemBytes = kSmemTop;        // enough for any start address of the window
+// Pipeline depth and X box stride by token tiles: four stages when the X boxes
+// (m <= 8 rows of 128 bytes) fit in 1 KB each, three otherwise.
+template <int kNT>
+struct GemvStages {
+  static constexpr int kStages = kNT == 1 ? 4 : 3;
+  static constexpr uint32_t kXBox = kNT == 1 ? 1024 : 2048;   // 1 KB aligned (128B swizzle)
+  static constexpr uint32_t kXTile = 4 * kXBox;
+  static constexpr uint32_t kSmemTop = kHighAddr + (kStages - 1) * kCodeTile;
+};
 
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   uint2 v;
@@ -165,6 +171,10 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
   constexpr int kWarps = S::kWarps;
   constexpr int kThreads = S::kThreads;
   constexpr int kRW = S::kRowsPerWarp;
+  constexpr int kStages = GemvStages<kNT>::kStages;
+  constexpr uint32_t kXBox = GemvStages<kNT>::kXBox;
+  constexpr uint32_t kXTile = GemvStages<kNT>::kXTile;
+  constexpr uint32_t kSmemTop = GemvStages<kNT>::kSmemTop;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw0 = smem_u32(smem_raw);
   uint32_t dyn_bytes;
@@ -327,22 +337,25 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
 
   if (threadIdx.x < 16) s_level[threadIdx.x] = a.level[threadIdx.x];
   __syncthreads();                        // levels, barrier initialisation
-  // pair table: entry (byte v, lane l) = {bf16(L[v >> 4]), bf16(L[v & 15])}, element order
-  for (int i = threadIdx.x; i < 256 * 32; i += kThreads) {
-    const int v = i >> 5, l = i & 31;
+  // pair table: entry (byte v, lane l) = {bf16(L[v >> 4]), bf16(L[v & 15])}, element order;
+  // thread v converts entry v once and writes its 32 copies
+  for (int v = threadIdx.x; v < 256; v += kThreads) {
     const __nv_bfloat162 e = __floats2bfloat162_rn(s_level[v >> 4], s_level[v & 15]);
-    sts32(kTableAddr + v * 256 + l * 4, *reinterpret_cast<const uint32_t*>(&e));
+    const float ev = __uint_as_float(*reinterpret_cast<const uint32_t*>(&e));
+#pragma unroll
+    for (int l = 0; l < 32; l += 4) sts128(kTableAddr + v * 256 + l * 4, ev, ev, ev, ev);
   }
   write_consts(pos, r0, 0);
   // X A^T over this CTA's 64-column blocks of K (blocks blockIdx.x + i * gridDim.x),
   // while the first code tiles are in flight.  The block's A slice [r x 64]
-  // goes to code stage 2 (not loaded before the main loop; chunk c of row j at
+  // goes to the last code stage (chunk c of row j at
   // ((c + j) mod 8) so that a quarter-warp reading chunk c of eight rows hits
   // distinct banks), its X slice [m x 64] to pair-table holes 64..79, and the
   // fp32 partial (m x r) stays in holes 128..255 until the end of the kernel.
+  // (The last code stage is first loaded in the main loop.)
   const int xa_n = m * a.r;                // <= 16 * 256 floats
   auto xa_hole = [](int e) { return hole(128u + (e >> 5), (e & 31) * 4u); };
-  const uint32_t a_stage = code_stage(2);
+  const uint32_t a_stage = code_stage(kStages - 1);
   for (int kb = blockIdx.x; kb < kblocks; kb += gridDim.x) {
     __syncthreads();                      // previous block's slices consumed
     for (int e = threadIdx.x; e < a.r * 8; e += kThreads) {
@@ -380,7 +393,7 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
       sts32(xa_hole(e), __float_as_uint(acc));
     }
   }
-  fence_proxy_async_smem();               // stage 2 is written by TMA from here on
+  fence_proxy_async_smem();               // the last stage is written by TMA from here on
   __syncthreads();                        // pair table, step 0's constants, X A^T partial in place
   launch_dependents();                    // k_finish may be scheduled; it waits for this grid
 
@@ -546,12 +559,15 @@ __global__ void __launch_bounds__(256) k_gemv_zero(float4* __restrict__ a, int64
   for (int64_t i = gtid; i < n4b; i += nthreads) b[i] = z;
 }
 
-// Y[i, n] = bf16(split[i, n] + s * sum_c XA[i, c] B[n, c]), one thread per row n.
+// Y[i, n] = bf16(split[i, n] + s * sum_c XA[i, c] B[n, c]).  Four lanes per
+// row n: lane q of the four takes the 8-column chunks cc = q, q + 4, ... of the
+// rank, the four partial sums are combined with two butterfly shuffles, and
+// lane q stores the tokens i = q, q + 4, ...
 __global__ void __launch_bounds__(128)
 k_finish(const float* __restrict__ yacc, const float* __restrict__ xa, int64_t ld_xa,
          const uint16_t* __restrict__ lora_b, int r, float s, int64_t m, int64_t nw, uint16_t* __restrict__ y,
          float* __restrict__ xa_out) {
-  __shared__ float s_xa[16 * 256];
+  __shared__ __align__(16) float s_xa[16 * 256];
   grid_dependency_wait();                  // k_gemv complete (it waited for k_gemv_zero)
   for (int e = threadIdx.x; e < m * r; e += blockDim.x) {
     const float v = __ldcg(xa + (e / r) * ld_xa + (e % r));
@@ -559,33 +575,50 @@ k_finish(const float* __restrict__ yacc, const float* __restrict__ xa, int64_t l
     if (xa_out && blockIdx.x == 0) xa_out[e] = v;
   }
   __syncthreads();
-  const int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (n >= nw) return;
+  const int q = threadIdx.x & 3;
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 4) + (threadIdx.x >> 2);
+  const bool live = n < nw;                // all lanes stay for the shuffles
   float lo[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) lo[i] = 0.0f;
-  const uint4* brow = reinterpret_cast<const uint4*>(lora_b + n * r);
-  for (int c0 = 0; c0 < r / 8; c0 += 8) {            // eight 16-byte loads in flight at a time
-    uint4 bv[8];
+  const uint4* brow = reinterpret_cast<const uint4*>(lora_b + (live ? n : 0) * r);
+  const int nch = r / 8;
+  for (int c0 = q; c0 < nch; c0 += 16) {   // up to four chunks in flight per lane
+    uint4 bv[4];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) bv[u] = (c0 + u < r / 8) ? __ldg(brow + c0 + u) : make_uint4(0u, 0u, 0u, 0u);
+    for (int u = 0; u < 4; ++u)
+      bv[u] = (live && c0 + 4 * u < nch) ? __ldg(brow + c0 + 4 * u) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (c0 + u >= r / 8) break;
-      const int cc = c0 + u;
+    for (int u = 0; u < 4; ++u) {
+      const int cc = c0 + 4 * u;
+      if (cc >= nch) break;
       const float b8[8] = {bf16_lo(bv[u].x), bf16_hi(bv[u].x), bf16_lo(bv[u].y), bf16_hi(bv[u].y),
                            bf16_lo(bv[u].z), bf16_hi(bv[u].z), bf16_lo(bv[u].w), bf16_hi(bv[u].w)};
 #pragma unroll
       for (int i = 0; i < 16; ++i)
         if (i < m) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) lo[i] = __fmaf_rn(s_xa[i * r + cc * 8 + e], b8[e], lo[i]);
+          const float4 x0 = *reinterpret_cast<const float4*>(&s_xa[i * r + cc * 8]);
+          const float4 x1 = *reinterpret_cast<const float4*>(&s_xa[i * r + cc * 8 + 4]);
+          float v = lo[i];
+          v = __fmaf_rn(x0.x, b8[0], v); v = __fmaf_rn(x0.y, b8[1], v);
+          v = __fmaf_rn(x0.z, b8[2], v); v = __fmaf_rn(x0.w, b8[3], v);
+          v = __fmaf_rn(x1.x, b8[4], v); v = __fmaf_rn(x1.y, b8[5], v);
+          v = __fmaf_rn(x1.z, b8[6], v); v = __fmaf_rn(x1.w, b8[7], v);
+          lo[i] = v;
         }
     }
   }
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     if (i < m) {
+      lo[i] += __shfl_xor_sync(0xFFFFFFFFu, lo[i], 1);
+      lo[i] += __shfl_xor_sync(0xFFFFFFFFu, lo[i], 2);
+    }
+  }
+  if (!live) return;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    if (i < m && (i & 3) == q) {
       const __nv_bfloat16 v = __float2bfloat16_rn(__fmaf_rn(s, lo[i], __ldcg(yacc + i * nw + n)));
       y[i * nw + n] = *reinterpret_cast<const uint16_t*>(&v);
     }
@@ -616,7 +649,7 @@ cudaError_t launch_gemv_t(const GemvArgs& args, const CUtensorMap& cm, const CUt
   const uint64_t bit = 1ull << (dev & 63);
   if (!(attr_done.load(std::memory_order_acquire) & bit)) {
     e = cudaFuncSetAttribute(k_gemv<kNT, kQuad, kMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes));
+                             static_cast<int>(GemvStages<kNT>::kSmemTop));
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(bit, std::memory_order_acq_rel);
   }
@@ -625,8 +658,9 @@ cudaError_t launch_gemv_t(const GemvArgs& args, const CUtensorMap& cm, const CUt
   GemvArgs a = args;
   CUtensorMap c = cm, x = xm;
   void* kargs[3] = {&a, &c, &x};
+  // dynamic shared memory up to the map's top covers any start address of the window
   return launch_pdl(reinterpret_cast<const void*>(k_gemv<kNT, kQuad, kMT>), dim3(grid),
-                    dim3(GemvShape<kMT>::kThreads), kSmemBytes, stream, kargs);
+                    dim3(GemvShape<kMT>::kThreads), GemvStages<kNT>::kSmemTop, stream, kargs);
 }
 
 template <int kMT>
@@ -666,7 +700,7 @@ cudaError_t launch_gemv(const GemvArgs& args, const CUtensorMap& codes_map, cons
 cudaError_t launch_gemv_finish(const float* yacc, const float* xa, int64_t ld_xa, const uint16_t* lora_b, int r,
                                float s, int64_t m, int64_t nw, uint16_t* y, float* xa_out, cudaStream_t stream) {
   void* kargs[10] = {&yacc, &xa, &ld_xa, &lora_b, &r, &s, &m, &nw, &y, &xa_out};
-  const unsigned grid = static_cast<unsigned>((nw + 127) / 128);
+  const unsigned grid = static_cast<unsigned>((nw + 31) / 32);      // 32 rows per 128-thread CTA
   return launch_pdl(reinterpret_cast<const void*>(k_finish), dim3(grid), dim3(128), 0, stream, kargs);
 }
 
