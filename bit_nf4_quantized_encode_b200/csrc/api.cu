@@ -306,6 +306,7 @@ qlora_status qlora_quantize_nf4_dq(const uint16_t* W, const qlora_nf4_tensor* ou
   for (int i = 0; i < kBuckets; ++i) {
     et.bucket_thr[i] = i < kNumBuckets ? tabs.bucket_thr[i] : INFINITY;
     et.bucket_base[i] = i < kNumBuckets ? tabs.bucket_base[i] : 15;
+    et.bucket_fast[i] = i < kNumBuckets ? tabs.bucket_fast[i] : (0x7F7FFFE0u | 16u);
   }
   et.fast = tabs.fast_ok ? 1 : 0;
 
@@ -315,7 +316,8 @@ qlora_status qlora_quantize_nf4_dq(const uint16_t* W, const qlora_nf4_tensor* ou
                                                round_up(static_cast<size_t>(nblocks) * 4, 256));
   const int64_t nvec = nblocks * 8;
   int grid = static_cast<int>((nvec + 255) / 256);
-  const int cap = d.num_sms * 8 < kMaxEncodeGrid ? d.num_sms * 8 : kMaxEncodeGrid;
+  const int wave = d.num_sms * encode_ctas_per_sm();           // one wave of resident CTAs
+  const int cap = wave < kMaxEncodeGrid ? wave : kMaxEncodeGrid;
   if (grid > cap) grid = cap;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = counted(launch_encode(W, numel, et, out->codes, c1buf, partials, grid, s));
@@ -340,7 +342,8 @@ qlora_status qlora_dequantize(const qlora_nf4_tensor* W, uint16_t* W_out, qlora_
   if ((st = device_info(&d)) != QLORA_OK) return st;
   const int64_t nchunks = (numel + 31) / 32;
   int grid = static_cast<int>((nchunks + 255) / 256);
-  if (grid > d.num_sms * 8) grid = d.num_sms * 8;
+  const int wave = d.num_sms * dequant_ctas_per_sm();          // one wave of resident CTAs
+  if (grid > wave) grid = wave;
   return cuda_status(counted(launch_dequant(W->codes, W->absmax_q, W->absmax_c2, W->absmax_mean,
                                             numel, codebook_param(), W_out, grid,
                                             reinterpret_cast<cudaStream_t>(stream))));

@@ -26,116 +26,159 @@
 namespace qlora {
 
 // ------------------------------------------------------------------ encode
-// One thread per 8 consecutive weights (one 16-byte load); 8 lanes form one
-// 64-weight block.  Writes packed codes, c1 per block, and one double partial
-// sum of c1 per CTA (for the tensor mean).  All 32 lanes of a warp execute
-// every shuffle; `mode` only changes how a lane loads and stores.
-enum : int { kVecNone = 0, kVecFull = 1, kVecTail = 2 };
+// Lanes 4j..4j+3 of a warp own one 64-weight block, 16 consecutive weights per
+// lane (two 16-byte loads, one 8-byte store of codes).  A CTA writes c1 per
+// block and one double partial sum of c1 (for the tensor mean).  Full blocks
+// go through the main loop; a ragged last block (numel not a multiple of 64)
+// is encoded by one thread afterwards.
+//
+// Fast path: n' = RN(x * RN(1/c1)) is within 2^-22 of the IEEE quotient
+// n = RN(x / c1) (three roundings of relative size 2^-24, |n| <= 1), so
+// code(n) == code(n') unless a threshold lies within 2^-22 of n'.  The bucket
+// of n' holds the only threshold that could (the table builder keeps every
+// threshold 2^-18 away from the bucket edges); its fast-path word carries that
+// threshold to within 2^-19 together with base + 1, and the code is
+// base + 1 - [n' < thr'].  When any element of the lane lands within 2^-18 of
+// its bucket's threshold (or is NaN), the lane redoes its 16 weights with IEEE
+// divisions and the exact table.
 
-__device__ __forceinline__ void encode_vec(const uint16_t* __restrict__ w, int64_t numel,
-                                           int64_t v, int mode, bool fast, const float* s_thr,
-                                           const uint8_t* s_base, uint8_t* __restrict__ codes,
-                                           float* __restrict__ c1buf, double& csum) {
-  float x[8];
-  const int64_t e0 = v * 8;
-  if (mode == kVecFull) {
-    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(w) + v);
-    x[0] = bf16_lo(raw.x); x[1] = bf16_hi(raw.x); x[2] = bf16_lo(raw.y); x[3] = bf16_hi(raw.y);
-    x[4] = bf16_lo(raw.z); x[5] = bf16_hi(raw.z); x[6] = bf16_lo(raw.w); x[7] = bf16_hi(raw.w);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      x[i] = (mode == kVecTail && e0 + i < numel)
-                 ? __uint_as_float(static_cast<uint32_t>(w[e0 + i]) << 16) : 0.0f;
-  }
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
-  // reduce over the 8 lanes of this block (lanes 8j..8j+7 of the warp)
-  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
-  if (mode == kVecNone) return;
+constexpr float kRiskBand = 0x1.0p-18f;
 
-  uint32_t packed = 0x77777777u;          // all zero-level codes
-  if (amax > 0.0f) {
-    // Fast path: n' = RN(x * RN(1/c1)) is within 2^-22 of the IEEE quotient
-    // RN(x / c1) (three roundings of relative size 2^-24, |n| <= 1), so its
-    // code equals the quotient's unless a threshold lies within 2^-22 of n'.
-    // The bucket of n' holds the only threshold that close (the table check
-    // keeps every threshold 2^-20 away from bucket edges); when n' is within
-    // 2^-20 of it the block's vector is redone with IEEE divisions.
-    bool exact = !fast || amax < 0x1.0p-125f;       // 1 / c1 must stay finite
-    if (!exact) {
-      const float r = __frcp_rn(amax);
-      uint32_t pk = 0;
-      bool risky = false;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float n = __fmul_rn(x[i], r);
-        const uint32_t u = __float_as_uint(__fmaf_rn(n, 16.0f, 8388624.0f)) & 63u;
-        const float d = __fsub_rn(n, s_thr[u]);     // exact sign; -inf when the bucket has no threshold
-        uint32_t code = s_base[u] + (d >= 0.0f ? 1u : 0u);
-        risky |= fabsf(d) <= 0x1.0p-20f;
-        if (mode == kVecTail && e0 + i >= numel) code = 7u;
-        pk |= code << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
-      }
-      if (risky) exact = true;
-      else packed = pk;
-    }
-    if (exact) {
-      packed = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float n = __fdiv_rn(x[i], amax);
-        // bucket u = RN(16 n + 16) via one fma against 2^23; then one compare
-        const uint32_t u = __float_as_uint(__fmaf_rn(n, 16.0f, 8388624.0f)) & 63u;
-        uint32_t code = s_base[u] + (n >= s_thr[u] ? 1u : 0u);
-        if (mode == kVecTail && e0 + i >= numel) code = 7u;
-        // element 2j -> high nibble of byte j, element 2j+1 -> low nibble
-        packed |= code << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
-      }
-    }
-  }
-  if (mode == kVecFull) {
-    reinterpret_cast<uint32_t*>(codes)[v] = packed;
-  } else {
-    const int64_t nbytes = (numel + 1) / 2;
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (v * 4 + j < nbytes) codes[v * 4 + j] = static_cast<uint8_t>(packed >> (8 * j));
-  }
-  if ((threadIdx.x & 7) == 0) {
-    c1buf[v >> 3] = amax;
-    csum += static_cast<double>(amax);
-  }
+// Exact code of n (float) from the exact bucket table.
+__device__ __forceinline__ uint32_t exact_code(float n, const float* s_thr, const uint8_t* s_base) {
+  const uint32_t u = __float_as_uint(__fmaf_rn(n, 16.0f, 8388624.0f)) & 63u;
+  return s_base[u] + (n >= s_thr[u] ? 1u : 0u);
+}
+
+__device__ __forceinline__ float nan_min_abs(float m, float d) {
+  float r;
+  asm("{\n\t.reg .f32 t;\n\tabs.f32 t, %2;\n\tmin.NaN.f32 %0, %1, t;\n\t}" : "=f"(r) : "f"(m), "f"(d));
+  return r;
 }
 
 __global__ void __launch_bounds__(256) k_encode(const uint16_t* __restrict__ w, int64_t numel,
                                                 EncodeTables tab, uint8_t* __restrict__ codes,
                                                 float* __restrict__ c1buf,
                                                 double* __restrict__ partials) {
+  __shared__ uint32_t s_fast[kBuckets];
   __shared__ float s_thr[kBuckets];
   __shared__ uint8_t s_base[kBuckets];
   __shared__ double s_red[8];
   for (int i = threadIdx.x; i < kBuckets; i += blockDim.x) {
+    s_fast[i] = tab.bucket_fast[i];
     s_thr[i] = tab.bucket_thr[i];
     s_base[i] = tab.bucket_base[i];
   }
   __syncthreads();
+  const uint32_t fast_tbl = static_cast<uint32_t>(__cvta_generic_to_shared(s_fast));
+  const bool fast_ok = tab.fast != 0;
 
-  // Vectors of 8 weights; a block of 64 is 8 vectors, i.e. 8 consecutive
-  // threads of one warp (the CTA size and grid stride are multiples of 8).
-  const int64_t nblocks = (numel + 63) / 64;
-  const int64_t nvec = nblocks * 8;                 // padded to whole blocks
-  const int64_t full_blocks = numel / 64;           // blocks with 64 real weights
+  const int64_t full_blocks = numel / 64;
+  const int64_t nq = full_blocks * 4;               // lane tasks of 16 weights
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const uint4* w4 = reinterpret_cast<const uint4*>(w);
   double csum = 0.0;
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x; base < nvec; base += stride) {
-    const int64_t v = base + threadIdx.x;
-    const int64_t blk = v >> 3;                     // the same for all 8 lanes of a group
-    const int mode = (blk < full_blocks) ? kVecFull : (blk < nblocks ? kVecTail : kVecNone);
-    encode_vec(w, numel, v, mode, tab.fast != 0, s_thr, s_base, codes, c1buf, csum);
+  // One task: 16 weights already loaded (r0, r1); lanes 4j..4j+3 share a block.
+  // Every lane executes the shuffles; `on` only gates the stores.
+  auto task = [&](int64_t v, bool on, const uint4 r0, const uint4 r1) {
+    const uint32_t wd[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+    float x[16];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      x[2 * k] = bf16_lo(wd[k]);
+      x[2 * k + 1] = bf16_hi(wd[k]);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+    if (!on) return;
+
+    uint32_t lo = 0x77777777u, hi = 0x77777777u;      // all zero-level codes
+    if (amax > 0.0f) {
+      // 1/c1 must be finite and c1 finite for the fast path
+      bool exact = !fast_ok || !(amax >= 0x1.0p-125f) || !(amax <= 3.0e38f);
+      if (!exact) {
+        const float r = __frcp_rn(amax);
+        float m = INFINITY;
+        uint32_t pk[2] = {0u, 0u};
+        // nibble order: element 2j -> high nibble of byte j; shift-add from byte 3 down
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int jj = 3; jj >= 0; --jj) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float n = __fmul_rn(x[8 * h + 2 * jj + e], r);
+              const uint32_t u = __float_as_uint(__fmaf_rn(n, 16.0f, 8388624.0f)) & 63u;
+              uint32_t tw;
+              asm("ld.shared.b32 %0, [%1];" : "=r"(tw) : "r"(fast_tbl + u * 4u));
+              const float d = __fsub_rn(n, __uint_as_float(tw));
+              m = nan_min_abs(m, d);
+              const uint32_t code = (tw & 31u) - (__float_as_uint(d) >> 31);
+              pk[h] = (pk[h] << 4) + code;
+            }
+          }
+        }
+        if (!(m > kRiskBand)) exact = true;
+        else { lo = pk[0]; hi = pk[1]; }
+      }
+      if (exact) {
+        uint32_t pk[2] = {0u, 0u};
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int jj = 3; jj >= 0; --jj)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+              pk[h] = (pk[h] << 4) + exact_code(__fdiv_rn(x[8 * h + 2 * jj + e], amax), s_thr, s_base);
+        lo = pk[0];
+        hi = pk[1];
+      }
+    }
+    reinterpret_cast<uint2*>(codes)[v] = make_uint2(lo, hi);
+    if ((threadIdx.x & 3) == 0) {
+      c1buf[v >> 2] = amax;
+      csum += static_cast<double>(amax);
+    }
+  };
+  // two tasks per iteration (a grid stride apart), both loaded before either is
+  // encoded; the loop bound is uniform over the CTA, so every lane reaches the
+  // shuffles
+  for (int64_t b0 = static_cast<int64_t>(blockIdx.x) * blockDim.x; b0 < nq; b0 += 2 * stride) {
+    const int64_t v0 = b0 + threadIdx.x, v1 = v0 + stride;
+    const bool on0 = v0 < nq, on1 = v1 < nq;
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    uint4 a0 = z, a1 = z, c0 = z, c1 = z;
+    if (on0) { a0 = __ldg(w4 + 2 * v0); a1 = __ldg(w4 + 2 * v0 + 1); }
+    if (on1) { c0 = __ldg(w4 + 2 * v1); c1 = __ldg(w4 + 2 * v1 + 1); }
+    task(v0, on0, a0, a1);
+    if (b0 + stride < nq) task(v1, on1, c0, c1);      // uniform over the CTA
+  }
+  // k_double_quant (launched as this grid's programmatic dependent) may now be
+  // scheduled; it waits for the whole grid before reading anything
+  asm volatile("griddepcontrol.launch_dependents;");
+  // ragged last block: one thread, exact path
+  if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0 && full_blocks * 64 < numel) {
+    const int64_t e0 = full_blocks * 64;
+    float amax = 0.0f;
+    for (int64_t e = e0; e < numel; ++e)
+      amax = fmaxf(amax, fabsf(__uint_as_float(static_cast<uint32_t>(w[e]) << 16)));
+    const int64_t nbytes = (numel + 1) / 2;
+    for (int64_t j = e0 / 2; j < nbytes; ++j) {
+      uint32_t c[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int64_t idx = 2 * j + e;
+        c[e] = 7u;
+        if (idx < numel && amax > 0.0f)
+          c[e] = exact_code(__fdiv_rn(__uint_as_float(static_cast<uint32_t>(w[idx]) << 16), amax), s_thr, s_base);
+      }
+      codes[j] = static_cast<uint8_t>((c[0] << 4) | c[1]);
+    }
+    c1buf[full_blocks] = amax;
+    csum += static_cast<double>(amax);
   }
   // deterministic per-CTA reduction of the partial sums
 #pragma unroll
@@ -157,6 +200,7 @@ __global__ void __launch_bounds__(256) k_double_quant(const float* __restrict__ 
                                                       int npartials, uint8_t* __restrict__ q,
                                                       float* __restrict__ c2, float* __restrict__ mean_out) {
   __shared__ double s_red[256];
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // k_encode complete
   double t = 0.0;
   for (int i = threadIdx.x; i < npartials; i += blockDim.x) t += partials[i];
   s_red[threadIdx.x] = t;
@@ -208,37 +252,82 @@ __global__ void __launch_bounds__(256) k_double_quant(const float* __restrict__ 
 }
 
 // ------------------------------------------------------------------ dequant
-// One thread per 32 codes (16 bytes in, 64 bytes out); a 64-weight block is
-// two threads.  Ragged tails fall back to element-wise work.
+// One lane per 32 codes (16 bytes in, 64 bytes out); a 64-weight block is two
+// lanes.  Each lane takes four chunks per iteration (a grid stride apart) and
+// issues the loads of all four before expanding any.  A ragged last chunk is
+// expanded element by element.
+__device__ __forceinline__ void dequant_chunk(const uint4 cw, uint32_t q, float c2v, float mu,
+                                              const CodebookParam& cb, uint4 (&o)[4]) {
+  const float c1p = block_constant(q, __fdiv_rn(c2v, 448.0f), mu);
+  const ByteTables t = make_tables(cb.level, c1p);
+  o[0] = expand8(cw.x, t);
+  o[1] = expand8(cw.y, t);
+  o[2] = expand8(cw.z, t);
+  o[3] = expand8(cw.w, t);
+}
+
+// The 32 lanes of a warp expand 32 consecutive chunks (2 KB of output).  Each
+// lane parks its 64 bytes in shared memory (rows of 80 bytes: conflict-free),
+// then the warp stores the 2 KB with every instruction covering 512
+// contiguous bytes.
 __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ codes,
                                                  const uint8_t* __restrict__ qabs,
                                                  const float* __restrict__ c2, const float* __restrict__ mean,
                                                  int64_t numel, CodebookParam cb,
                                                  uint16_t* __restrict__ out) {
+  __shared__ __align__(16) uint8_t s_out[8][32 * 80];
   const float mu = __ldg(mean);
-  const int64_t nchunks = (numel + 31) / 32;
+  const int64_t nfull = numel / 32;                  // chunks of 32 real weights
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t ch = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; ch < nchunks;
-       ch += stride) {
-    const int64_t blk = ch >> 1;
-    const float c2v = __ldg(c2 + (blk >> 8));
-    const float c1p = block_constant(__ldg(qabs + blk), __fdiv_rn(c2v, 448.0f), mu);
-    const ByteTables t = make_tables(cb.level, c1p);
-    const int64_t e0 = ch * 32;
-    if (e0 + 32 <= numel) {
-      const uint4 cw = __ldg(reinterpret_cast<const uint4*>(codes) + ch);
-      uint4* dst = reinterpret_cast<uint4*>(out + e0);
-      dst[0] = expand8(cw.x, t);
-      dst[1] = expand8(cw.y, t);
-      dst[2] = expand8(cw.z, t);
-      dst[3] = expand8(cw.w, t);
-    } else {
-      for (int64_t e = e0; e < numel; ++e) {
-        const uint32_t byte = codes[e >> 1];
-        const uint32_t code = (e & 1) ? (byte & 15u) : (byte >> 4);
-        const __nv_bfloat16 v = __float2bfloat16_rn(__fmul_rn(cb.level[code], c1p));
-        out[e] = *reinterpret_cast<const uint16_t*>(&v);
+  const uint4* cw4 = reinterpret_cast<const uint4*>(codes);
+  uint4* out4 = reinterpret_cast<uint4*>(out);
+  const int lane = threadIdx.x & 31;
+  uint8_t* st = s_out[threadIdx.x >> 5];
+  // the loop bound is uniform over the CTA, so every lane reaches the syncwarps
+  for (int64_t b0 = static_cast<int64_t>(blockIdx.x) * blockDim.x; b0 < nfull; b0 += 4 * stride) {
+    const int64_t ch = b0 + threadIdx.x;
+    uint4 cw[4];
+    uint32_t qv[4];
+    float c2v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t c = ch + u * stride;
+      cw[u] = make_uint4(0u, 0u, 0u, 0u);
+      qv[u] = 0;
+      c2v[u] = 0.0f;
+      if (c < nfull) {
+        cw[u] = __ldg(cw4 + c);
+        qv[u] = __ldg(qabs + (c >> 1));
+        c2v[u] = __ldg(c2 + (c >> 9));
       }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t c = ch + u * stride;
+      const int64_t wc0 = c - lane;                  // the warp's first chunk
+      uint4 o[4];
+      dequant_chunk(cw[u], qv[u], c2v[u], mu, cb, o);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4*>(st + lane * 80 + k * 16) = o[k];
+      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int p = lane + 32 * j;                 // 16-byte piece of the warp's 2 KB
+        const int src = p >> 2;                      // the lane that expanded it
+        if (wc0 + src < nfull) out4[wc0 * 4 + p] = *reinterpret_cast<const uint4*>(st + src * 80 + (p & 3) * 16);
+      }
+      __syncwarp();
+    }
+  }
+  // ragged last chunk
+  if (blockIdx.x == 0 && threadIdx.x == 0 && nfull * 32 < numel) {
+    const int64_t blk = nfull >> 1;
+    const float c1p = block_constant(qabs[blk], __fdiv_rn(c2[blk >> 8], 448.0f), mu);
+    for (int64_t e = nfull * 32; e < numel; ++e) {
+      const uint32_t byte = codes[e >> 1];
+      const uint32_t code = (e & 1) ? (byte & 15u) : (byte >> 4);
+      const __nv_bfloat16 v = __float2bfloat16_rn(__fmul_rn(cb.level[code], c1p));
+      out[e] = *reinterpret_cast<const uint16_t*>(&v);
     }
   }
 }
@@ -253,8 +342,29 @@ cudaError_t launch_encode(const uint16_t* w, int64_t numel, const EncodeTables& 
 cudaError_t launch_double_quant(const float* c1buf, int64_t nblocks, const double* partials,
                                 int npartials, uint8_t* q, float* c2, float* mean, int grid,
                                 cudaStream_t stream) {
-  k_double_quant<<<grid, 256, 0, stream>>>(c1buf, nblocks, partials, npartials, q, c2, mean);
-  return cudaGetLastError();
+  // programmatic dependent of k_encode: the launch overlaps the encoder's tail
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_double_quant, c1buf, nblocks, partials, npartials, q, c2, mean);
+}
+
+int dequant_ctas_per_sm() {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_dequant, 256, 0) != cudaSuccess || n < 1) n = 1;
+  return n;
+}
+
+int encode_ctas_per_sm() {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_encode, 256, 0) != cudaSuccess || n < 1) n = 1;
+  return n;
 }
 
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* qabs, const float* c2,

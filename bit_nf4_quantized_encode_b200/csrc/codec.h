@@ -10,9 +10,10 @@ namespace qlora {
 // Buckets 33..63 are padding (never reached for finite inputs).
 constexpr int kBuckets = 64;
 struct EncodeTables {
-  float bucket_thr[kBuckets];
-  uint8_t bucket_base[kBuckets];
-  int fast;                  // nonzero: the reciprocal path of the encoder may be used
+  float bucket_thr[kBuckets];       // exact path: the threshold inside bucket u (or +inf)
+  uint8_t bucket_base[kBuckets];    // exact path: code of the smallest n in bucket u
+  uint32_t bucket_fast[kBuckets];   // fast path: threshold bits with base + 1 in the low 5 bits
+  int fast;                         // nonzero: the reciprocal path may be used
 };
 
 // The 16 NF4 levels, passed by value.
@@ -22,6 +23,11 @@ struct CodebookParam {
 
 cudaError_t launch_encode(const uint16_t* w, int64_t numel, const EncodeTables& tab, uint8_t* codes,
                           float* c1buf, double* partials, int grid, cudaStream_t stream);
+// Resident k_encode / k_dequant CTAs per SM (their grids are one wave of them).
+int encode_ctas_per_sm();
+int dequant_ctas_per_sm();
+// k_double_quant is launched as the programmatic dependent of k_encode, which
+// must be the kernel before it in the stream.
 cudaError_t launch_double_quant(const float* c1buf, int64_t nblocks, const double* partials,
                                 int npartials, uint8_t* q, float* c2, float* mean, int grid,
                                 cudaStream_t stream);

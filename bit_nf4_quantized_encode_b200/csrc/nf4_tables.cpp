@@ -112,12 +112,16 @@ Nf4Tables build() {
     }
     if (inside > 1) t.ok = false;
     // The encoder's reciprocal path only re-checks the threshold of the bucket
-    // its estimate falls in; that is exact when no threshold is within 2^-20
-    // of a bucket edge (the estimate is within 2^-22 of the IEEE quotient).
-    if (inside == 1 && (static_cast<double>(thr) - nlo <= 0x1.0p-20 || nhi - static_cast<double>(thr) <= 0x1.0p-20))
+    // its estimate falls in; that is exact when no threshold is within 2^-18
+    // of a bucket edge (the estimate is within 2^-22 of the IEEE quotient, and
+    // the fast-path threshold within 2^-19 of the true one).
+    if (inside == 1 && (static_cast<double>(thr) - nlo <= 0x1.0p-18 || nhi - static_cast<double>(thr) <= 0x1.0p-18))
       t.fast_ok = false;
     t.bucket_base[u] = static_cast<uint8_t>(base);
     t.bucket_thr[u] = thr;
+    uint32_t tb = 0x7F7FFFE0u;                 // about 3.4e38: no threshold in this bucket
+    if (inside == 1) std::memcpy(&tb, &thr, 4);
+    t.bucket_fast[u] = (tb & ~31u) | static_cast<uint32_t>(base + 1);
   }
   return t;
 }

@@ -14,8 +14,12 @@ struct Nf4Tables {
   float threshold[15];        // code(n) = #{i : n >= threshold[i]}
   float bucket_thr[kNumBuckets];     // the one threshold inside bucket u, or +inf
   uint8_t bucket_base[kNumBuckets];  // code of the smallest n in bucket u
+  // Fast-path word of bucket u: the threshold's float bits with the low five
+  // mantissa bits replaced by bucket_base[u] + 1 (a bucket without a threshold
+  // gets a huge finite float); the perturbation is below 2^-19.
+  uint32_t bucket_fast[kNumBuckets];
   bool ok;                    // every bucket holds at most one threshold
-  bool fast_ok;               // every threshold lies more than 2^-20 inside its bucket
+  bool fast_ok;               // every threshold lies more than 2^-18 inside its bucket
 };
 
 // Built once (thread-safe) on first use.

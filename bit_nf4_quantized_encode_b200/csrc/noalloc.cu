@@ -95,6 +95,7 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const uint16_t* W, const q
   for (int i = 0; i < kBuckets; ++i) {
     et.bucket_thr[i] = i < kNumBuckets ? tabs.bucket_thr[i] : INFINITY;
     et.bucket_base[i] = i < kNumBuckets ? tabs.bucket_base[i] : 15;
+    et.bucket_fast[i] = i < kNumBuckets ? tabs.bucket_fast[i] : (0x7F7FFFE0u | 16u);
   }
   et.fast = tabs.fast_ok ? 1 : 0;
 
@@ -102,7 +103,8 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const uint16_t* W, const q
   float* c1buf = static_cast<float*>(scratch);
   double* partials = reinterpret_cast<double*>(static_cast<unsigned char*>(scratch) + kNoAllocC1Bytes);
   int grid = static_cast<int>((nblocks * 8 + 255) / 256);
-  const int cap = num_sms * 8 < kNoAllocPartials ? num_sms * 8 : kNoAllocPartials;
+  const int wave = num_sms * encode_ctas_per_sm();             // one wave of resident CTAs
+  const int cap = wave < kNoAllocPartials ? wave : kNoAllocPartials;
   if (grid > cap) grid = cap;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (launch_encode(W, numel, et, out->codes, c1buf, partials, grid, s) != cudaSuccess)

@@ -110,6 +110,40 @@ def test_codec_thresholds_and_levels(qb):
     _assert_codec_equal(qb, w)
 
 
+def _near_threshold_pairs(band=2.0 ** -18):
+    """(c1, x) bf16 pairs whose IEEE quotient x / c1 lies within `band` of a
+    decision midpoint, found by search over c1 (CPU, float32 arithmetic)."""
+    L = oracle.codebook().astype(np.float64)
+    mids = [(L[i] + L[i + 1]) / 2 for i in range(15)]
+    # positive bf16 values with exponents 2^-6 .. 2^6
+    c1 = oracle.bf16_bits_to_f32(np.arange(0x3C80, 0x4300, dtype=np.uint16))
+    pairs = []
+    for mid in mids:
+        t = oracle.bf16_rne_array((c1 * np.float32(mid)).astype(np.float32))
+        for delta in (-1, 0, 1):
+            xb = (t.astype(np.int32) + (delta if mid >= 0 else -delta)).astype(np.uint16)
+            x = oracle.bf16_bits_to_f32(xb)
+            q = (x / c1).astype(np.float32)                 # IEEE float division
+            hit = np.abs(q.astype(np.float64) - mid) <= band
+            hit &= np.abs(x) <= c1
+            pairs += list(zip(c1[hit], x[hit]))
+    return pairs
+
+
+def test_codec_quotients_next_to_thresholds(qb):
+    """Blocks whose element quotient falls within 2^-18 of a decision midpoint:
+    the encoder's reciprocal path must hand these to the IEEE-division path."""
+    pairs = _near_threshold_pairs()
+    assert len(pairs) >= 20, len(pairs)
+    blocks = []
+    for c1, x in pairs:
+        blk = np.zeros(64, np.float32)
+        blk[0], blk[17], blk[38], blk[63] = c1, x, -x, np.float32(0.5) * x
+        blocks.append(blk)
+    w = torch.from_numpy(np.concatenate(blocks)).to(torch.bfloat16).reshape(len(pairs), 64)
+    _assert_codec_equal(qb, w)
+
+
 def test_codec_zero_and_constant_blocks(qb):
     w = torch.zeros(4, 512, dtype=torch.bfloat16)
     w[1, :] = 0.5                      # constant blocks: c2 may be zero in a group
