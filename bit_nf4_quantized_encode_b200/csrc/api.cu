@@ -122,6 +122,18 @@ bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t oute
   return r == CUDA_SUCCESS;
 }
 
+// m-tiles per rasterization group of the fused kernel: the packed codes of one
+// group (128 rows or columns of W times `contraction` weights, half a byte
+// each) should take about 48 MB, so that they stay in the 126 MB L2 while the
+// group sweeps the token tiles.
+int m_group_for(int m_tiles, int64_t contraction) {
+  const int64_t per_tile = 64 * contraction;
+  int64_t g = (int64_t{48} << 20) / (per_tile > 0 ? per_tile : 1);
+  if (g < 1) g = 1;
+  if (g > m_tiles) g = m_tiles;
+  return static_cast<int>(g);
+}
+
 // Split count for `tiles` output tiles of `ksteps` steps each over `sms` CTAs:
 // minimises the makespan ceil(tiles * s / sms) * ceil(ksteps / s), counting two
 // steps of fixed cost per work unit.
@@ -452,6 +464,7 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor* W, const uint16_t* X, int6
   fa.m_tiles = static_cast<int>((sh.rows + 127) / 128);
   fa.t_tiles = static_cast<int>((sh.m + bn - 1) / bn);
   fa.splits = 1;
+  fa.m_group = m_group_for(fa.m_tiles, sh.cols);
   fa.out = Y; fa.out_acc = nullptr;
   fa.cb = codebook_param();
   fa.err = d.err;
@@ -530,6 +543,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor* W, const uint16_t* X, cons
     fa.m_tiles = static_cast<int>((sh.cols + 127) / 128);
     fa.t_tiles = static_cast<int>((sh.m + bn - 1) / bn);
     fa.splits = sh.decode ? choose_splits(fa.m_tiles, fa.ksteps, d.num_sms) : 1;
+    fa.m_group = m_group_for(fa.m_tiles, sh.rows);
     fa.out = dX; fa.out_acc = dx_acc;
     fa.cb = codebook_param();
     fa.err = d.err;

@@ -41,20 +41,28 @@ __host__ __device__ constexpr size_t fused_smem_bytes(int bn) {
   return 1024 + static_cast<size_t>(fused_stages(bn)) * (kATileBytes + bn * 128) + 512;
 }
 
-// Work unit -> (m-tile, token tile, split) and its k-step range.
+// Work unit -> (m-tile, token tile, split) and its k-step range.  Units run in
+// groups of m_group m-tiles: inside a group the m-tile varies fastest (after the
+// split) and the group sweeps every token tile before the next group starts, so
+// the codes of one group (a few tens of MB) stay in L2 while every token tile
+// re-reads them, and a token tile of activations is reused by the whole group.
 struct Unit {
   int mt, tt, sp;
   int kbeg, kmain;     // first main k-step, number of main k-steps
   int nk;              // main + LoRA k-steps
 };
 
-__device__ __forceinline__ Unit decode_unit(int u, int m_tiles, int splits, int ksteps,
-                                            int lora_steps) {
+__device__ __forceinline__ Unit decode_unit(int u, int m_tiles, int t_tiles, int m_group, int splits,
+                                            int ksteps, int lora_steps) {
   Unit w;
   w.sp = u % splits;
   const int rest = u / splits;
-  w.mt = rest % m_tiles;
-  w.tt = rest / m_tiles;
+  const int per_group = m_group * t_tiles;
+  const int gi = rest / per_group;
+  const int r2 = rest - gi * per_group;
+  const int gsz = min(m_group, m_tiles - gi * m_group);      // the last group may be short
+  w.mt = gi * m_group + r2 % gsz;
+  w.tt = r2 / gsz;
   w.kbeg = static_cast<int>((static_cast<int64_t>(ksteps) * w.sp) / splits);
   const int kend = static_cast<int>((static_cast<int64_t>(ksteps) * (w.sp + 1)) / splits);
   w.kmain = kend - w.kbeg;
@@ -67,10 +75,17 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
                "r"(v.w) : "memory");
 }
 
-__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+// L2 policy for the packed codes: every token tile of a launch re-reads the
+// whole weight, so it is kept in L2 ahead of the streamed output.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p, uint64_t pol) {
   uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p), "l"(pol));
   return v;
 }
 
@@ -83,7 +98,7 @@ struct DqLoad {
 };
 
 template <int kDir>
-__device__ __forceinline__ DqLoad dq_load(const FusedArgs& a, int m0, int kstep, int t) {
+__device__ __forceinline__ DqLoad dq_load(const FusedArgs& a, int m0, int kstep, int t, uint64_t pol) {
   DqLoad d;
   int64_t n, kcol;
   if (kDir == 0) {              // forward: task = W row m0 + t, block kstep
@@ -97,8 +112,8 @@ __device__ __forceinline__ DqLoad dq_load(const FusedArgs& a, int m0, int kstep,
   if (d.valid) {
     const int64_t e = n * a.kw + kcol;                 // first weight of the block
     const uint8_t* p = a.codes + (e >> 1);
-    d.c0 = ldg_nc_v4(p);
-    d.c1 = ldg_nc_v4(p + 16);
+    d.c0 = ldg_nc_v4(p, pol);
+    d.c1 = ldg_nc_v4(p + 16, pol);
     const int64_t blk = e >> 6;
     d.q = __ldg(a.qabs + blk);
     d.c2 = __ldg(a.c2 + (blk >> 8));
@@ -218,19 +233,20 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
     const int group = warp >> 2;              // warps 4g .. 4g+3
     const int t = threadIdx.x & 127;
     const float mu = __ldg(a.mean);
+    const uint64_t codes_pol = l2_evict_last_policy();
     uint32_t gctr = 0;
     bool alive = true;
     for (int u = blockIdx.x; u < nunits && alive; u += gridDim.x) {
-      const Unit w = decode_unit(u, a.m_tiles, a.splits, a.ksteps, a.lora_steps);
+      const Unit w = decode_unit(u, a.m_tiles, a.t_tiles, a.m_group, a.splits, a.ksteps, a.lora_steps);
       const int m0 = w.mt * 128;
       int j = static_cast<int>((static_cast<uint32_t>(group) - gctr) & (kDequantGroups - 1));
       DqLoad next;
-      if (j < w.kmain) next = dq_load<kDir>(a, m0, w.kbeg + j, t);
+      if (j < w.kmain) next = dq_load<kDir>(a, m0, w.kbeg + j, t, codes_pol);
       for (; j < w.nk; j += kDequantGroups) {
         const uint32_t it = gctr + j;
         const uint32_t stage = it % kStages, phase = (it / kStages) & 1u;
         const DqLoad cur = next;
-        if (j + kDequantGroups < w.kmain) next = dq_load<kDir>(a, m0, w.kbeg + j + kDequantGroups, t);
+        if (j + kDequantGroups < w.kmain) next = dq_load<kDir>(a, m0, w.kbeg + j + kDequantGroups, t, codes_pol);
         if (!mbar_wait(&empty[stage], phase ^ 1u, a.err)) { alive = false; break; }
         const uint32_t sA = smem0 + stage * kStageBytes;
         if (j < w.kmain) dq_store<kDir>(sA, t, cur, mu, a.cb);
@@ -246,7 +262,7 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
       uint32_t gctr = 0;
       bool alive = true;
       for (int u = blockIdx.x; u < nunits && alive; u += gridDim.x) {
-        const Unit w = decode_unit(u, a.m_tiles, a.splits, a.ksteps, a.lora_steps);
+        const Unit w = decode_unit(u, a.m_tiles, a.t_tiles, a.m_group, a.splits, a.ksteps, a.lora_steps);
         for (int j = 0; j < w.nk; ++j) {
           const uint32_t it = gctr + j;
           const uint32_t stage = it % kStages, phase = (it / kStages) & 1u;
@@ -267,7 +283,7 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
       uint32_t gctr = 0, uctr = 0;
       bool alive = true;
       for (int u = blockIdx.x; u < nunits && alive; u += gridDim.x, ++uctr) {
-        const Unit w = decode_unit(u, a.m_tiles, a.splits, a.ksteps, a.lora_steps);
+        const Unit w = decode_unit(u, a.m_tiles, a.t_tiles, a.m_group, a.splits, a.ksteps, a.lora_steps);
         const uint32_t ab = uctr & 1u, aphase = (uctr >> 1) & 1u;
         if (!mbar_wait(&acc_empty[ab], aphase ^ 1u, a.err)) break;
         tc_fence_after();
@@ -300,7 +316,7 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
     const int quarter = warp & 3;             // the four epilogue warps cover lane quarters 0..3
     uint32_t uctr = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++uctr) {
-      const Unit w = decode_unit(u, a.m_tiles, a.splits, a.ksteps, a.lora_steps);
+      const Unit w = decode_unit(u, a.m_tiles, a.t_tiles, a.m_group, a.splits, a.ksteps, a.lora_steps);
       const uint32_t ab = uctr & 1u, aphase = (uctr >> 1) & 1u;
       if (!mbar_wait(&acc_full[ab], aphase, a.err)) break;
       tc_fence_after();
@@ -329,7 +345,7 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
               atomicAdd(a.out_acc + tok * a.ldo + row, val);
             } else {
               const __nv_bfloat16 b = __float2bfloat16_rn(val);
-              a.out[tok * a.ldo + row] = *reinterpret_cast<const uint16_t*>(&b);
+              __stcs(a.out + tok * a.ldo + row, *reinterpret_cast<const unsigned short*>(&b));   // streamed out
             }
           }
         }

@@ -39,6 +39,7 @@ struct FusedArgs {
   int64_t mdim;              // MMA-M extent: fwd nw, bwd kw
   int ksteps;                // main k-steps: contraction / 64 (rounded up)
   int m_tiles, t_tiles, splits;
+  int m_group;               // m-tiles swept across all token tiles before the next group
   CodebookParam cb;
   uint32_t* err;             // device error flag
 };
