@@ -562,32 +562,55 @@ __global__ void __launch_bounds__(256) k_gemv_zero(float4* __restrict__ a, int64
 // Y[i, n] = bf16(split[i, n] + s * sum_c XA[i, c] B[n, c]).  Four lanes per
 // row n: lane q of the four takes the 8-column chunks cc = q, q + 4, ... of the
 // rank, the four partial sums are combined with two butterfly shuffles, and
-// lane q stores the tokens i = q, q + 4, ...
+// lane q stores the tokens i = q, q + 4, ...  kMaxM (1, 4, 8 or 16) bounds the
+// token count at compile time.
+template <int kMaxM>
 __global__ void __launch_bounds__(128)
 k_finish(const float* __restrict__ yacc, const float* __restrict__ xa, int64_t ld_xa,
          const uint16_t* __restrict__ lora_b, int r, float s, int64_t m, int64_t nw, uint16_t* __restrict__ y,
          float* __restrict__ xa_out) {
-  __shared__ __align__(16) float s_xa[16 * 256];
+  __shared__ __align__(16) float s_xa[kMaxM * 256];
   grid_dependency_wait();                  // k_gemv complete (it waited for k_gemv_zero)
-  for (int e = threadIdx.x; e < m * r; e += blockDim.x) {
-    const float v = __ldcg(xa + (e / r) * ld_xa + (e % r));
-    s_xa[e] = v;
-    if (xa_out && blockIdx.x == 0) xa_out[e] = v;
+  const int mi = static_cast<int>(m);
+  // X A^T into shared memory (row i at i * r)
+  for (int j = threadIdx.x; j < r; j += blockDim.x) {
+    float v[kMaxM];
+#pragma unroll
+    for (int i = 0; i < kMaxM; ++i) v[i] = i < mi ? __ldcg(xa + i * ld_xa + j) : 0.0f;
+#pragma unroll
+    for (int i = 0; i < kMaxM; ++i)
+      if (i < mi) {
+        s_xa[i * r + j] = v[i];
+        if (xa_out && blockIdx.x == 0) xa_out[i * r + j] = v[i];
+      }
   }
-  __syncthreads();
   const int q = threadIdx.x & 3;
   const int64_t n = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 4) + (threadIdx.x >> 2);
   const bool live = n < nw;                // all lanes stay for the shuffles
-  float lo[16];
+  // split-buffer values of this lane's tokens and its first B chunks are issued
+  // before the barrier, with the staging loads: one memory round trip per row
+  constexpr int kMine = (kMaxM + 3) / 4;   // tokens stored by this lane
+  float acc[kMine];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) lo[i] = 0.0f;
+  for (int u = 0; u < kMine; ++u) {
+    const int i = q + 4 * u;
+    acc[u] = (live && i < mi) ? __ldcg(yacc + i * nw + n) : 0.0f;
+  }
   const uint4* brow = reinterpret_cast<const uint4*>(lora_b + (live ? n : 0) * r);
   const int nch = r / 8;
-  for (int c0 = q; c0 < nch; c0 += 16) {   // up to four chunks in flight per lane
-    uint4 bv[4];
+  uint4 bv[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      bv[u] = (live && c0 + 4 * u < nch) ? __ldg(brow + c0 + 4 * u) : make_uint4(0u, 0u, 0u, 0u);
+  for (int u = 0; u < 4; ++u) bv[u] = (live && q + 4 * u < nch) ? __ldg(brow + q + 4 * u) : make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();                         // X A^T staged
+  float lo[kMaxM];
+#pragma unroll
+  for (int i = 0; i < kMaxM; ++i) lo[i] = 0.0f;
+  for (int c0 = q; c0 < nch; c0 += 16) {   // four chunks of eight rank columns per round
+    if (c0 != q) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        bv[u] = (live && c0 + 4 * u < nch) ? __ldg(brow + c0 + 4 * u) : make_uint4(0u, 0u, 0u, 0u);
+    }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int cc = c0 + 4 * u;
@@ -595,8 +618,8 @@ k_finish(const float* __restrict__ yacc, const float* __restrict__ xa, int64_t l
       const float b8[8] = {bf16_lo(bv[u].x), bf16_hi(bv[u].x), bf16_lo(bv[u].y), bf16_hi(bv[u].y),
                            bf16_lo(bv[u].z), bf16_hi(bv[u].z), bf16_lo(bv[u].w), bf16_hi(bv[u].w)};
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        if (i < m) {
+      for (int i = 0; i < kMaxM; ++i)
+        if (i < mi) {
           const float4 x0 = *reinterpret_cast<const float4*>(&s_xa[i * r + cc * 8]);
           const float4 x1 = *reinterpret_cast<const float4*>(&s_xa[i * r + cc * 8 + 4]);
           float v = lo[i];
@@ -609,18 +632,21 @@ k_finish(const float* __restrict__ yacc, const float* __restrict__ xa, int64_t l
     }
   }
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    if (i < m) {
-      lo[i] += __shfl_xor_sync(0xFFFFFFFFu, lo[i], 1);
-      lo[i] += __shfl_xor_sync(0xFFFFFFFFu, lo[i], 2);
-    }
+  for (int i = 0; i < kMaxM; ++i) {
+    lo[i] += __shfl_xor_sync(0xFFFFFFFFu, lo[i], 1);
+    lo[i] += __shfl_xor_sync(0xFFFFFFFFu, lo[i], 2);
   }
   if (!live) return;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    if (i < m && (i & 3) == q) {
-      const __nv_bfloat16 v = __float2bfloat16_rn(__fmaf_rn(s, lo[i], __ldcg(yacc + i * nw + n)));
-      y[i * nw + n] = *reinterpret_cast<const uint16_t*>(&v);
+  for (int u = 0; u < kMine; ++u) {
+    const int i = q + 4 * u;
+    float v = lo[0];                         // lo[i] with compile-time indices
+#pragma unroll
+    for (int k = 1; k < kMaxM; ++k)
+      if (k == i) v = lo[k];
+    if (i < mi) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(__fmaf_rn(s, v, acc[u]));
+      y[i * nw + n] = *reinterpret_cast<const uint16_t*>(&h);
     }
   }
 }
@@ -701,7 +727,11 @@ cudaError_t launch_gemv_finish(const float* yacc, const float* xa, int64_t ld_xa
                                float s, int64_t m, int64_t nw, uint16_t* y, float* xa_out, cudaStream_t stream) {
   void* kargs[10] = {&yacc, &xa, &ld_xa, &lora_b, &r, &s, &m, &nw, &y, &xa_out};
   const unsigned grid = static_cast<unsigned>((nw + 31) / 32);      // 32 rows per 128-thread CTA
-  return launch_pdl(reinterpret_cast<const void*>(k_finish), dim3(grid), dim3(128), 0, stream, kargs);
+  const void* fn = m <= 1 ? reinterpret_cast<const void*>(k_finish<1>)
+                 : m <= 4 ? reinterpret_cast<const void*>(k_finish<4>)
+                 : m <= 8 ? reinterpret_cast<const void*>(k_finish<8>)
+                          : reinterpret_cast<const void*>(k_finish<16>);
+  return launch_pdl(fn, dim3(grid), dim3(128), 0, stream, kargs);
 }
 
 }  // namespace qlora
