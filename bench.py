@@ -47,6 +47,28 @@ def load_peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
+def fused_traffic():
+    """DRAM bytes (read + written) of one k_fused launch of the headline step,
+    from the committed ncu summary -- or None when that summary was not taken
+    on the fused kernel's current source (its sha256 is recorded with it)."""
+    import hashlib
+    summary = os.path.join(ROOT, "profiles", "k_fused_dram_traffic_llama65b_m8192.md")
+    src = os.path.join(ROOT, "bit_nf4_quantized_encode_b200", "csrc", "gemm.cu")
+    try:
+        with open(src, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+        recorded, traffic = None, None
+        with open(summary) as f:
+            for line in f:
+                if line.startswith("source_sha256"):
+                    recorded = line.split(":", 1)[1].strip()
+                elif line.startswith("traffic_bytes_per_launch:"):
+                    traffic = int(line.split(":", 1)[1].strip())
+    except (OSError, ValueError):
+        return None
+    return traffic if recorded == digest else None
+
+
 # ---------------------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
@@ -406,7 +428,8 @@ def bench_ours(args):
         "roofline": {"bound": "tensor", "kernel": "k_fused (dequant-GEMM fwd and bwd-dX)",
                      "achieved": round(achieved, 1), "peak": peak_t, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_t, 4), "peak_kind": f"{peak_kind} sustained bf16",
-                     "traffic": None, "avg_launch_ms": round(fused_avg_s * 1e3, 4),
+                     "traffic": fused_traffic(), "traffic_unit": "bytes per launch (ncu, profiles/)",
+                     "avg_launch_ms": round(fused_avg_s * 1e3, 4),
                      "share_of_step": round(sum(gemm_ms) / 1e3 / t_local, 4)},
         "clocks": clk,
     }
