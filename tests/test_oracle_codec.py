@@ -225,7 +225,7 @@ def test_storage_golden_matches_pages():
     assert g["bits_without_dq"] - g["bits_with_dq_asymptotic"] == g["bits_saved_asymptotic"]
     assert round(g["bits_saved_asymptotic"], 2) == g["bits_saved_pages_approx"]
     gb = g["params_65b"] * g["bits_saved_asymptotic"] / 8 / 1e9
-    assert round(gb) == g["gb_saved_65b_pages_approx"]        # "roughly 3 GB on a 65B model"
+    assert round(gb) == g["gb_saved_65b_pages_approx"]        # the pages' approximate figure for 65B
     # count the real bytes for a 65B-parameter tensor (a multiple of 64*256)
     numel = int(g["params_65b"]) // 16384 * 16384
     sb = oracle.storage_bytes(numel)
