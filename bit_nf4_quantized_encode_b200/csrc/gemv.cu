@@ -5,14 +5,13 @@
 // weight is dequantized on the fly for the matmul), bound by HBM.  Three
 // kernels, each launched as the programmatic dependent of the one before it:
 //
-// k_gemv_zero: zeroes the fp32 accumulators of k_gemv (split buffer, X A^T).
+// k_xa_zero: partial X A^T over slices of K in fp32 (CUDA cores, CTAs that fit
+//   beside k_gemv's) and the zeroed fp32 split buffer of k_gemv.
 //
 // k_gemv: the weight stream.  Each CTA takes an equal, contiguous share of all
 //   (256-row tile, 256-column step) pairs, so the work is balanced whatever the
 //   shape; a CTA adds its fp32 partial of each tile it touched to the split
-//   buffer with atomics.  While its first loads are in flight, each CTA also
-//   computes X A^T over its share of the 64-column blocks of K (fp32, CUDA
-//   cores) and adds it to the X A^T accumulator at its end.
+//   buffer with atomics, and at its end sums its share of the X A^T slices.
 //   * Thread 0 streams the [256 rows x 128 bytes] code tile (128B-swizzled) and
 //     the four [m x 64] activation boxes of each step into a 3-deep ring (TMA).
 //   * 16 / kMT warps own 16 kMT weight rows each.  For every 64-column block
@@ -240,14 +239,13 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
     return true;
   };
   if (producer) {
-    // barriers first, then the first loads: they are in flight while the
-    // pair table is built
+    tma_prefetch_desc(&cmap);
+    tma_prefetch_desc(&xmap);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], kWarps);
     }
     fence_barrier_init();
-    for (int i = 0; i < kStages - 1; ++i) issue_next(true);
   }
 
   // ------------------------------------------------ compute
@@ -337,6 +335,9 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
 
   if (threadIdx.x < 16) s_level[threadIdx.x] = a.level[threadIdx.x];
   __syncthreads();                        // levels, barrier initialisation
+  // the first loads are in flight while the pair table is built
+  if (producer)
+    for (int i = 0; i < kStages - 1; ++i) issue_next(true);
   // pair table: entry (byte v, lane l) = {bf16(L[v >> 4]), bf16(L[v & 15])}, element order;
   // thread v converts entry v once and writes its 32 copies
   for (int v = threadIdx.x; v < 256; v += kThreads) {
@@ -346,55 +347,7 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
     for (int l = 0; l < 32; l += 4) sts128(kTableAddr + v * 256 + l * 4, ev, ev, ev, ev);
   }
   write_consts(pos, r0, 0);
-  // X A^T over this CTA's 64-column blocks of K (blocks blockIdx.x + i * gridDim.x),
-  // while the first code tiles are in flight.  The block's A slice [r x 64]
-  // goes to the last code stage (chunk c of row j at
-  // ((c + j) mod 8) so that a quarter-warp reading chunk c of eight rows hits
-  // distinct banks), its X slice [m x 64] to pair-table holes 64..79, and the
-  // fp32 partial (m x r) stays in holes 128..255 until the end of the kernel.
-  // (The last code stage is first loaded in the main loop.)
-  const int xa_n = m * a.r;                // <= 16 * 256 floats
-  auto xa_hole = [](int e) { return hole(128u + (e >> 5), (e & 31) * 4u); };
-  const uint32_t a_stage = code_stage(kStages - 1);
-  for (int kb = blockIdx.x; kb < kblocks; kb += gridDim.x) {
-    __syncthreads();                      // previous block's slices consumed
-    for (int e = threadIdx.x; e < a.r * 8; e += kThreads) {
-      const int j = e >> 3, ch = e & 7;
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.lora_a + static_cast<int64_t>(j) * a.kw + kb * 64) + ch);
-      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_stage + j * 128u + ((ch + j) & 7) * 16u),
-                   "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
-    }
-    for (int e = threadIdx.x; e < m * 8; e += kThreads) {
-      const int i = e >> 3, ch = e & 7;
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<int64_t>(i) * a.kw + kb * 64) + ch);
-      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(hole(64u + i, ch * 16u)),
-                   "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < xa_n; e += kThreads) {
-      const int i = e / a.r, j = e % a.r;
-      float acc = kb == static_cast<int>(blockIdx.x) ? 0.0f : __uint_as_float(lds_table(xa_hole(e)));
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        uint4 av, xv;
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(av.x), "=r"(av.y), "=r"(av.z), "=r"(av.w)
-                     : "r"(a_stage + j * 128u + ((ch + j) & 7) * 16u));
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(xv.x), "=r"(xv.y), "=r"(xv.z), "=r"(xv.w)
-                     : "r"(hole(64u + i, ch * 16u)));
-        acc = __fmaf_rn(bf16_lo(av.x), bf16_lo(xv.x), acc);
-        acc = __fmaf_rn(bf16_hi(av.x), bf16_hi(xv.x), acc);
-        acc = __fmaf_rn(bf16_lo(av.y), bf16_lo(xv.y), acc);
-        acc = __fmaf_rn(bf16_hi(av.y), bf16_hi(xv.y), acc);
-        acc = __fmaf_rn(bf16_lo(av.z), bf16_lo(xv.z), acc);
-        acc = __fmaf_rn(bf16_hi(av.z), bf16_hi(xv.z), acc);
-        acc = __fmaf_rn(bf16_lo(av.w), bf16_lo(xv.w), acc);
-        acc = __fmaf_rn(bf16_hi(av.w), bf16_hi(xv.w), acc);
-      }
-      sts32(xa_hole(e), __float_as_uint(acc));
-    }
-  }
-  fence_proxy_async_smem();               // the last stage is written by TMA from here on
-  __syncthreads();                        // pair table, step 0's constants, X A^T partial in place
+  __syncthreads();                        // pair table and step 0's constants in place
   launch_dependents();                    // k_finish may be scheduled; it waits for this grid
 
   // X rows of this lane (token 8n + g); lanes of tokens >= m load nothing, and
@@ -417,8 +370,8 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
       for (int e = 0; e < 4; ++e) y[i][n][e] = 0.0f;
   // The partial of the first tile this CTA touches is kept in registers until
   // the next tile boundary (or the end of the range): by then the previous
-  // kernel (zeroing of the accumulators) has surely finished, so the wait for
-  // it does not stall the stream.
+  // kernel (X A^T and the zeroed split buffer) has surely finished, so the wait
+  // for it does not stall the stream.
   float ys[kMT][kNT][4];
   int ys_tile = -1;
   bool dep_done = false;
@@ -539,24 +492,95 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
     if (++s == kStages) { s = 0; ph ^= 1u; }
   }
   if (!alive) return;
-  if (blockIdx.x < kblocks) {
-    if (!dep_done) grid_dependency_wait();
-    for (int e = threadIdx.x; e < xa_n; e += kThreads)
-      atomicAdd(a.xa + (e / a.r) * a.ld_xa + (e % a.r), __uint_as_float(lds_table(xa_hole(e))));
+  // this CTA's share of X A^T: the sum of k_xa_zero's K slices (complete once
+  // the wait above has returned; every CTA reached it at its last flush)
+  {
+    const int nxa = m * a.r;
+    const int e_beg = static_cast<int>((static_cast<int64_t>(nxa) * blockIdx.x) / gridDim.x);
+    const int e_end = static_cast<int>((static_cast<int64_t>(nxa) * (blockIdx.x + 1)) / gridDim.x);
+    for (int e = e_beg + static_cast<int>(threadIdx.x); e < e_end; e += kThreads) {
+      const int i = e / a.r, j = e - (e / a.r) * a.r;
+      float v = 0.0f;
+      for (int sp = 0; sp < a.xa_splits; ++sp) v += __ldcg(a.xa_part + (static_cast<int64_t>(sp) * 16 + i) * a.ld_xa + j);
+      a.xa[i * a.ld_xa + j] = v;
+    }
   }
 }
 
-// Zeroes the accumulators of k_gemv.  k_gemv is launched as its programmatic
-// dependent: it starts streaming the weight at once and waits for this grid
-// only before its first atomic.
-__global__ void __launch_bounds__(256) k_gemv_zero(float4* __restrict__ a, int64_t n4a, float4* __restrict__ b,
-                                                   int64_t n4b) {
+// Partial X A^T and the zeroed split buffer of k_gemv.  CTA (c, sp) computes
+// LoRA columns 4c .. 4c + 3 for every token over the sp-th of nsplit slices of
+// K and writes them to part[sp] (no atomics, so nothing needs zeroing); k_gemv
+// sums the slices at its end.  Each of the 64 threads takes 8-column chunks a
+// block stride apart; the CTA reduces with warp shuffles and one exchange
+// through shared memory.  64 threads of at most 128 registers, so that a CTA
+// fits beside a k_gemv CTA on one SM: k_gemv, launched as the programmatic
+// dependent of this grid, starts streaming at once and only waits for it
+// before its first atomic.
+template <int kMaxM>
+__global__ void __launch_bounds__(64, 8)
+k_xa_zero(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A, int64_t m, int64_t kw, int r,
+          float* __restrict__ part, int64_t ld, float4* __restrict__ zero4, int64_t n4) {
   launch_dependents();
-  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  __shared__ float s_red[4 * kMaxM];
+  const int mi = static_cast<int>(m);
+  const int j0 = blockIdx.x * 4;
+  const int64_t nch = kw / 8;
+  const int64_t c_beg = (nch * blockIdx.y) / gridDim.y, c_end = (nch * (blockIdx.y + 1)) / gridDim.y;
+  float acc[4][kMaxM];
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+#pragma unroll
+    for (int i = 0; i < kMaxM; ++i) acc[c][i] = 0.0f;
+  for (int64_t ch = c_beg + threadIdx.x; ch < c_end; ch += blockDim.x) {
+    float af[4][8];                        // the four A rows' 8 columns, unpacked once
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 v = (j0 + c < r) ? __ldg(reinterpret_cast<const uint4*>(A + (j0 + c) * kw) + ch)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+      af[c][0] = bf16_lo(v.x); af[c][1] = bf16_hi(v.x); af[c][2] = bf16_lo(v.y); af[c][3] = bf16_hi(v.y);
+      af[c][4] = bf16_lo(v.z); af[c][5] = bf16_hi(v.z); af[c][6] = bf16_lo(v.w); af[c][7] = bf16_hi(v.w);
+    }
+    uint4 xv[kMaxM];
+#pragma unroll
+    for (int i = 0; i < kMaxM; ++i)
+      xv[i] = i < mi ? __ldg(reinterpret_cast<const uint4*>(X + i * kw) + ch) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int i = 0; i < kMaxM; ++i) {
+      const float xf[8] = {bf16_lo(xv[i].x), bf16_hi(xv[i].x), bf16_lo(xv[i].y), bf16_hi(xv[i].y),
+                           bf16_lo(xv[i].z), bf16_hi(xv[i].z), bf16_lo(xv[i].w), bf16_hi(xv[i].w)};
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[c][i] = __fmaf_rn(af[c][e], xf[e], acc[c][i]);
+    }
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+#pragma unroll
+    for (int i = 0; i < kMaxM; ++i) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[c][i] += __shfl_xor_sync(0xFFFFFFFFu, acc[c][i], o);
+    }
+  if (warp == 1 && lane == 0) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int i = 0; i < kMaxM; ++i) s_red[c * kMaxM + i] = acc[c][i];
+  }
+  __syncthreads();
+  if (warp == 0 && lane == 0) {
+    float* dst = part + static_cast<int64_t>(blockIdx.y) * 16 * ld;
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int i = 0; i < kMaxM; ++i)
+        if (i < mi && j0 + c < r) dst[i * ld + j0 + c] = acc[c][i] + s_red[c * kMaxM + i];
+  }
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * gridDim.y * blockDim.x;
+  const int64_t gtid = (static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x;
   const float4 z = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  for (int64_t i = gtid; i < n4a; i += nthreads) a[i] = z;
-  for (int64_t i = gtid; i < n4b; i += nthreads) b[i] = z;
+  for (int64_t e = gtid; e < n4; e += nthreads) zero4[e] = z;
 }
 
 // Y[i, n] = bf16(split[i, n] + s * sum_c XA[i, c] B[n, c]).  Four lanes per
@@ -570,7 +594,7 @@ k_finish(const float* __restrict__ yacc, const float* __restrict__ xa, int64_t l
          const uint16_t* __restrict__ lora_b, int r, float s, int64_t m, int64_t nw, uint16_t* __restrict__ y,
          float* __restrict__ xa_out) {
   __shared__ __align__(16) float s_xa[kMaxM * 256];
-  grid_dependency_wait();                  // k_gemv complete (it waited for k_gemv_zero)
+  grid_dependency_wait();                  // k_gemv complete (it waited for k_xa_zero)
   const int mi = static_cast<int>(m);
   // X A^T into shared memory (row i at i * r)
   for (int j = threadIdx.x; j < r; j += blockDim.x) {
@@ -704,14 +728,25 @@ cudaError_t launch_gemv_mt(const GemvArgs& args, const CUtensorMap& cm, const CU
 
 int gemv_tile_rows() { return kRows; }
 
-cudaError_t launch_gemv_zero(float* a, int64_t n_a, float* b, int64_t n_b, cudaStream_t stream) {
-  const int64_t n4 = (n_a > n_b ? n_a : n_b) / 4;
-  int64_t grid = (n4 + 255) / 256;
-  if (grid > 1024) grid = 1024;
-  if (grid < 1) grid = 1;
-  k_gemv_zero<<<static_cast<unsigned>(grid), 256, 0, stream>>>(reinterpret_cast<float4*>(a), n_a / 4,
-                                                               reinterpret_cast<float4*>(b), n_b / 4);
+cudaError_t launch_xa_zero(const uint16_t* X, const uint16_t* A, int64_t m, int64_t kw, int r, float* part,
+                           int64_t ld, int splits, float* zero, int64_t n_zero, cudaStream_t stream) {
+  const dim3 grid(static_cast<unsigned>((r + 3) / 4), static_cast<unsigned>(splits));
+  float4* z4 = reinterpret_cast<float4*>(zero);
+  const int64_t n4 = n_zero / 4;
+  if (m <= 1) k_xa_zero<1><<<grid, 64, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4);
+  else if (m <= 4) k_xa_zero<4><<<grid, 64, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4);
+  else if (m <= 8) k_xa_zero<8><<<grid, 64, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4);
+  else k_xa_zero<16><<<grid, 64, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4);
   return cudaGetLastError();
+}
+
+int xa_splits_for(int r, int64_t kw) {
+  const int groups = (r + 3) / 4;
+  int s = 128 / groups;                       // about 128 CTAs in all
+  const int64_t max_by_k = (kw / 8) / 64;     // at least one chunk per thread
+  if (s > max_by_k) s = static_cast<int>(max_by_k);
+  if (s > kMaxXaSplits) s = kMaxXaSplits;
+  return s < 1 ? 1 : s;
 }
 
 cudaError_t launch_gemv(const GemvArgs& args, const CUtensorMap& codes_map, const CUtensorMap& x_map,

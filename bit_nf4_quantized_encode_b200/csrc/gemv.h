@@ -13,12 +13,12 @@ struct GemvArgs {
   const float* mean;         // per-tensor mean
   int64_t nw, kw;            // W shape (rows = out features, cols = in features)
   int64_t m;                 // token rows (<= 16)
-  float* yacc;               // fp32 [m, nw] accumulator, zeroed by k_gemv_zero
-  const uint16_t* x;         // X bf16 [m, kw]
-  const uint16_t* lora_a;    // LoRA A bf16 [r, kw]
-  float* xa;                 // fp32 [m, ld_xa] accumulator of X A^T, zeroed by k_gemv_zero
+  float* yacc;               // fp32 [m, nw] accumulator, zeroed by k_xa_zero
+  const float* xa_part;      // k_xa_zero's X A^T slices: [xa_splits][16][ld_xa] fp32
+  float* xa;                 // X A^T [m, ld_xa] fp32, summed by k_gemv at its end
   int64_t ld_xa;
-  int r;
+  int r;                     // LoRA rank
+  int xa_splits;
   int m_tiles;               // tiles of gemv_tile_rows() weight rows
   int steps;                 // 256-column steps per row
   float level[16];           // NF4 levels
@@ -27,13 +27,19 @@ struct GemvArgs {
 
 int gemv_tile_rows();
 
-// Zeroes the two fp32 accumulators of k_gemv (n_a and n_b floats, multiples of 4).
-cudaError_t launch_gemv_zero(float* a, int64_t n_a, float* b, int64_t n_b, cudaStream_t stream);
+// Upper bound on the K slices of X A^T (the work buffer holds that many).
+constexpr int kMaxXaSplits = 16;
+// K slices of X A^T for rank r and contraction kw (1 .. kMaxXaSplits).
+int xa_splits_for(int r, int64_t kw);
+// Partial X A^T (fp32 [splits][16][ld]) for m <= 16 tokens, and the zeroing of
+// zero[n_zero] (k_gemv's split buffer; n_zero a multiple of 4, 16-byte aligned).
+cudaError_t launch_xa_zero(const uint16_t* X, const uint16_t* A, int64_t m, int64_t kw, int r, float* part,
+                           int64_t ld, int splits, float* zero, int64_t n_zero, cudaStream_t stream);
 
 // codes_map: packed codes as uint8 [nw, kw/2], box {128, 256}, 128-byte swizzle.
 // x_map: X bf16 [m, kw], box {64, m}, 128-byte swizzle.
 // k_gemv is launched as a programmatic dependent of the kernel before it in the
-// stream, which must be k_gemv_zero of the same call.
+// stream, which must be k_xa_zero of the same call.
 cudaError_t launch_gemv(const GemvArgs& args, const CUtensorMap& codes_map, const CUtensorMap& x_map,
                         int num_sms, cudaStream_t stream);
 
