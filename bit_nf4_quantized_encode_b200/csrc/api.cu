@@ -195,14 +195,16 @@ qlora_status check_linear(const qlora_nf4_tensor* W, int64_t M, int32_t r, Linea
 // Work buffer layout: fp32 accumulators first (one memset clears them all),
 // then bf16 staging.  Offsets in bytes, each 256-aligned.
 struct FwdLayout {
-  size_t xa_acc, y_acc, fp32_end, sxa, xa_part, xa_slices, total;
+  size_t xa_acc, cnt, slots, fp32_end, sxa, xa_slices, total;
 };
 FwdLayout fwd_layout(const LinearShape& s) {
   FwdLayout l{};
   size_t o = 0;
-  if (s.decode) {        // k_xa_zero + k_gemv + k_finish: split buffer, X A^T
-    l.y_acc = o;    o = round_up(o + size_t(s.m) * s.rows * 4, 256);
-    l.xa_part = o;  o = round_up(o + size_t(16) * s.rpad * 4, 256);
+  if (s.decode) {        // k_xa_zero + k_gemv: tile counters, partial slots, X A^T slices
+    const size_t m_tiles = (size_t(s.rows) + gemv_tile_rows() - 1) / gemv_tile_rows();
+    const size_t steps = (size_t(s.cols) / 64 + 3) / 4;
+    l.cnt = o;      o = round_up(o + m_tiles * 8 * 4, 256);
+    l.slots = o;    o = round_up(o + size_t(gemv_slot_floats(int64_t(m_tiles), int64_t(steps))) * 4, 256);
     l.xa_slices = o; o = round_up(o + size_t(kMaxXaSplits) * 16 * s.rpad * 4, 256);
     l.fp32_end = 0;
     l.total = o;
@@ -400,16 +402,16 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor* W, const uint16_t* X, int6
   uint8_t* ws = static_cast<uint8_t*>(workspace);
 
   if (sh.decode) {
-    // Decode shapes: X A^T and the zeroed split buffer (k_xa_zero), one pass
-    // over the packed weight (k_gemv), then Y with the LoRA term (k_finish);
-    // each kernel is the programmatic dependent of the one before.
-    float* y_acc = reinterpret_cast<float*>(ws + L.y_acc);
-    float* xa = reinterpret_cast<float*>(ws + L.xa_part);
+    // Decode shapes: X A^T slices and the zeroed tile counters (k_xa_zero),
+    // then one pass over the packed weight that also writes Y (k_gemv, the
+    // programmatic dependent of k_xa_zero).
+    uint32_t* cnt = reinterpret_cast<uint32_t*>(ws + L.cnt);
     const int m_tiles = static_cast<int>((sh.rows + gemv_tile_rows() - 1) / gemv_tile_rows());
     float* xa_slices = reinterpret_cast<float*>(ws + L.xa_slices);
     const int xa_splits = xa_splits_for(sh.r, sh.cols);
-    if (counted(launch_xa_zero(X, A, sh.m, sh.cols, sh.r, xa_slices, sh.rpad, xa_splits, y_acc, sh.m * sh.rows,
-                               cs)) != cudaSuccess)
+    if (counted(launch_xa_zero(X, A, sh.m, sh.cols, sh.r, xa_slices, sh.rpad, xa_splits,
+                               reinterpret_cast<float*>(cnt), static_cast<int64_t>(m_tiles) * 8, cs)) !=
+        cudaSuccess)
       return QLORA_ERR_CUDA;
     CUtensorMap c_map, x_act;
     if (!make_map_u8(&c_map, W->codes, sh.cols / 2, sh.rows, sh.cols / 2, 128, gemv_tile_rows(),
@@ -419,16 +421,17 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor* W, const uint16_t* X, int6
     GemvArgs ga{};
     ga.qabs = W->absmax_q; ga.c2 = W->absmax_c2; ga.mean = W->absmax_mean;
     ga.nw = sh.rows; ga.kw = sh.cols; ga.m = sh.m;
-    ga.yacc = y_acc;
-    ga.xa_part = xa_slices; ga.xa = xa; ga.ld_xa = sh.rpad; ga.r = sh.r; ga.xa_splits = xa_splits;
+    ga.slots = reinterpret_cast<float*>(ws + L.slots);
+    ga.cnt = cnt;
+    ga.xa_part = xa_slices; ga.ld_xa = sh.rpad; ga.r = sh.r; ga.lora_steps = sh.lora_steps;
+    ga.xa_splits = xa_splits;
+    ga.s = s; ga.lora_b = B; ga.y = Y; ga.xa_out = XA_out;
     ga.m_tiles = m_tiles;
     ga.steps = static_cast<int>((sh.cols / 64 + 3) / 4);
     const CodebookParam cbp = codebook_param();
     for (int i = 0; i < 16; ++i) ga.level[i] = cbp.level[i];
     ga.err = d.err;
     if (counted(launch_gemv(ga, c_map, x_act, d.num_sms, cs)) != cudaSuccess) return QLORA_ERR_CUDA;
-    if (counted(launch_gemv_finish(y_acc, xa, sh.rpad, B, sh.r, s, sh.m, sh.rows, Y, XA_out, cs)) != cudaSuccess)
-      return QLORA_ERR_CUDA;
     return QLORA_OK;
   }
 

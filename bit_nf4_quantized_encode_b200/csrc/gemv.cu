@@ -2,32 +2,37 @@
 //
 // Y = X deq(W)^T + s (X A^T) B^T with few token rows is a stream over the packed
 // weight (automatone "QLoRA paper explained", section "How it works": the 4-bit
-// weight is dequantized on the fly for the matmul), bound by HBM.  Three
-// kernels, each launched as the programmatic dependent of the one before it:
+// weight is dequantized on the fly for the matmul), bound by HBM.  Two kernels,
+// the second launched as the programmatic dependent of the first:
 //
 // k_xa_zero: partial X A^T over slices of K in fp32 (CUDA cores, CTAs that fit
-//   beside k_gemv's) and the zeroed fp32 split buffer of k_gemv.
+//   beside k_gemv's), and the zeroed fp32 split buffer and tile counters of
+//   k_gemv.
 //
-// k_gemv: the weight stream.  Each CTA takes an equal, contiguous share of all
-//   (256-row tile, 256-column step) pairs, so the work is balanced whatever the
-//   shape; a CTA adds its fp32 partial of each tile it touched to the split
-//   buffer with atomics, and at its end sums its share of the X A^T slices.
-//   * Thread 0 streams the [256 rows x 128 bytes] code tile (128B-swizzled) and
-//     the four [m x 64] activation boxes of each step into a 3-deep ring (TMA).
-//   * 16 / kMT warps own 16 kMT weight rows each.  For every 64-column block
+// k_gemv: the weight stream and the whole output.  Each CTA takes an equal,
+//   contiguous share of all (256-row tile, 256-column step) pairs, so the work
+//   is balanced whatever the shape.
+//   * A producer warp streams the [256 rows x 128 bytes] code tile
+//     (128B-swizzled) and the four [m x 64] activation boxes of each step into
+//     a 3- or 4-deep ring (TMA), and writes the step's block constants
+//     c1' = fma(e4m3(q), c2/448, mu) into the stage.
+//   * Eight consumer warps own 32 weight rows each.  For every 64-column block
 //     they read their rows' code bytes, turn each byte into the two bf16 levels
 //     it encodes with one shared-memory load from a 256-entry pair table (one
 //     copy per lane: conflict-free), and feed them straight from registers to
 //     warp MMAs (m16n8k16, bf16 in, fp32 out): a code byte is exactly one
-//     A-fragment register.  The block's product is scaled by its constant
-//     c1' = fma(e4m3(q), c2/448, mu) and added to fp32 registers.
+//     A-fragment register.  The block's product is scaled by its constant and
+//     added to fp32 registers.
+//   * A tile shared by several CTAs is summed in an fp32 split buffer; the warp
+//     whose partial completes a tile's 32 rows (a per-warp counter) adds the
+//     LoRA up-projection with warp MMAs over the staged bf16(s X A^T) and
+//     writes those rows of Y.  A tile inside one CTA's share is finished from
+//     registers.
 //   * The tensor core here only replaces FMAs: per weight it does 2 M FLOP.
 //     Warp MMAs are used because a skinny-N product issued as tcgen05.mma
 //     from one thread costs about 80 cycles per 128x16x16 instruction, which
 //     caps a 16-token stream near 25 weights per cycle per SM, while HBM
 //     delivers about 46.
-//
-// k_finish: Y = bf16(split + s (X A^T) B^T), one thread per weight row.
 //
 // Numerics: the block constant multiplies the fp32 product of its block, so a
 // weight enters as bf16(L[code]) * c1' rather than bf16(L[code] * c1'): the same
@@ -89,9 +94,6 @@ __device__ __forceinline__ uint32_t lds_table(uint32_t addr) {
   asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
 }
-__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
 __device__ __forceinline__ void sts128(uint32_t addr, float a, float b, float c, float d) {
   asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
@@ -132,6 +134,14 @@ __device__ __forceinline__ void e4m3x4_to_f32(uint32_t q, float (&f)[4]) {
   f[2] = __half2float(__ushort_as_half(static_cast<unsigned short>(hi & 0xFFFFu)));
   f[3] = __half2float(__ushort_as_half(static_cast<unsigned short>(hi >> 16)));
 }
+// Named barriers: 1 between the producer warps (arrive, do not wait) and the
+// consumer warps (wait for all `count` threads); 2 among the producer warps.
+__device__ __forceinline__ void named_barrier_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
@@ -143,6 +153,10 @@ __device__ __forceinline__ void launch_dependents() {
 __device__ __forceinline__ int64_t bound(int i, int64_t total, int ctas) {
   return (static_cast<int64_t>(i) * total) / ctas;
 }
+// The CTA whose share holds global step u (ctas <= total, so no share is empty).
+__device__ __forceinline__ int64_t owner_of(int64_t u, int64_t total, int ctas) {
+  return ((u + 1) * ctas - 1) / total;
+}
 
 // Block-constant inputs of one step for one weight row, loaded ahead: the E4M3
 // bytes of the step's four blocks (byte b = block b) and c2 of the first
@@ -153,23 +167,22 @@ struct RowConsts {
   float c2a, c2b;
 };
 
-// kMT m16 tiles (16 kMT weight rows) per warp, 16 / kMT warps per CTA.
-template <int kMT>
-struct GemvShape {
-  static constexpr int kWarps = 16 / kMT;
-  static constexpr int kThreads = kWarps * 32;
-  static constexpr int kRowsPerWarp = 16 * kMT;
-  static constexpr int kMaxRegs = kMT == 1 ? 112 : 224;
-};
+// Eight consumer warps own 32 weight rows each (two m16 MMA tiles); warps
+// 8..11 are producers, one per SM sub-partition, so that their work weighs on
+// all four schedulers alike.  Each sub-partition then holds three warps:
+// 3 x 32 x 168 registers fit its 16K.
+constexpr int kConsumerWarps = 8;
+constexpr int kProducerWarps = 4;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kGemvThreads = kConsumers + kProducerWarps * 32;
+constexpr int kGemvMaxRegs = 168;
+constexpr int kRowsPerProducerLane = kRows / (kProducerWarps * 32);
+constexpr uint32_t kSxaHole = 128;     // first pair-table hole row of the s X A^T staging
 
-template <int kNT, bool kQuad, int kMT>   // kNT: n8 token tiles (1: M <= 8, 2: M <= 16); kQuad: K % 256 == 0
-__global__ void __maxnreg__(GemvShape<kMT>::kMaxRegs)
+template <int kNT, bool kQuad>   // kNT: n8 token tiles (1: M <= 8, 2: M <= 16); kQuad: K % 256 == 0
+__global__ void __maxnreg__(kGemvMaxRegs)
 k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
        const __grid_constant__ CUtensorMap xmap) {
-  using S = GemvShape<kMT>;
-  constexpr int kWarps = S::kWarps;
-  constexpr int kThreads = S::kThreads;
-  constexpr int kRW = S::kRowsPerWarp;
   constexpr int kStages = GemvStages<kNT>::kStages;
   constexpr uint32_t kXBox = GemvStages<kNT>::kXBox;
   constexpr uint32_t kXTile = GemvStages<kNT>::kXTile;
@@ -188,17 +201,19 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
   auto gptr = [&](uint32_t addr) { return smem_raw + (addr - raw0); };
   auto code_stage = [&](uint32_t s) { return s == 0 ? cs_low : kHighAddr + (s - 1) * kCodeTile; };
   uint64_t* bars = reinterpret_cast<uint64_t*>(gptr(misc));
-  uint64_t* full = bars;                  // codes + X landed (TMA)
-  uint64_t* empty = bars + kStages;       // one arrival per warp
-  float* s_level = reinterpret_cast<float*>(gptr(misc + 64));
+  uint64_t* full = bars;                  // codes + X landed (TMA) and constants written (producer)
+  uint64_t* empty = bars + kStages;       // one arrival per consumer warp
+  uint64_t* xa_bar = bars + 2 * kStages;  // s X A^T staged (one arrival per consumer warp)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t steps = a.steps;
   const int64_t total = static_cast<int64_t>(a.m_tiles) * steps;
-  const int64_t x_beg = bound(blockIdx.x, total, gridDim.x);
-  const int64_t x_end = bound(blockIdx.x + 1, total, gridDim.x);
+  const int ctas = static_cast<int>(gridDim.x);
+  const int64_t x_beg = bound(blockIdx.x, total, ctas);
+  const int64_t x_end = bound(blockIdx.x + 1, total, ctas);
   const int kblocks = static_cast<int>(a.kw / 64);
+  const uint32_t kbl = static_cast<uint32_t>(kblocks);
   const int m = static_cast<int>(a.m);
 
   // Position of a step: (tile, step within the tile's row of steps).  Advanced
@@ -213,142 +228,145 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
   const int64_t n_mine = x_end - x_beg;
   const Pos first{static_cast<int>(x_beg / steps), static_cast<int>(x_beg % steps)};
 
-  // TMA issue (thread 0): iteration i goes to stage i % kStages once every warp
-  // has released that stage's previous iteration.
-  const uint32_t xbytes = 4u * static_cast<uint32_t>(m) * 128u;
-  const bool producer = threadIdx.x == 0;
-  Pos ppos = first;
-  int64_t pit = 0;
-  uint32_t ps = 0, pph = 0;
-  // issue the next step if its stage is free; `block` waits (bounded) for it
-  auto issue_next = [&](bool block) -> bool {
-    if (pit >= n_mine) return true;
-    if (!mbar_test_wait(&empty[ps], pph ^ 1u)) {
-      if (!block) return true;
-      if (!mbar_wait(&empty[ps], pph ^ 1u, a.err)) return false;
-    }
-    mbar_arrive_expect_tx(&full[ps], kCodeTile + xbytes);
-    const int col0 = ppos.step * kStepCols;
-    tma_load_2d(gptr(code_stage(ps)), &cmap, col0 / 2, ppos.tile * kRows, &full[ps]);
-#pragma unroll
-    for (int b = 0; b < 4; ++b)
-      tma_load_2d(gptr(xs0 + ps * kXTile + b * kXBox), &xmap, col0 + b * 64, 0, &full[ps]);
-    ppos = advance(ppos);
-    ++pit;
-    if (++ps == kStages) { ps = 0; pph ^= 1u; }
-    return true;
-  };
-  if (producer) {
+  // Block constants of step p for tile rows lane + 32 j (j < 8), staged in the
+  // free halves of the pair-table rows: slot s holds row r's four constants at
+  // hole(32 s + r / 8, 16 (r mod 8)).
+  if (threadIdx.x == kConsumers) {
     tma_prefetch_desc(&cmap);
     tma_prefetch_desc(&xmap);
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kWarps);
+      mbar_init(&full[i], 1 + kProducerWarps);
+      mbar_init(&empty[i], kConsumerWarps);
     }
+    mbar_init(xa_bar, kConsumerWarps);
     fence_barrier_init();
   }
-
-  // ------------------------------------------------ compute
-  // Lane (g, t) serves MMA rows g and g + 8 of the warp's kMT m16 tiles.  MMA
-  // row g of an 8-row group is weight row 8u + pg with pg = 2(g mod 4) + g / 4,
-  // so that the lanes of each half-warp read rows whose 128-byte swizzle
-  // patterns differ in bits 1 and 2 (no bank conflicts).  The lane's rows are
-  // warp*16kMT + 8q + pg (q < 2kMT; tile i uses q = 2i and 2i + 1).  In every
-  // 64-column block the lane reads the code bytes [8t, 8t + 8) of those rows.
-  // Columns enter the MMA in a permuted order (the same for X): slice j of a
-  // block feeds columns 16t + 4j + {0, 1} as k = {2t, 2t+1} and 16t + 4j + {2, 3}
-  // as k = {2t+8, 2t+9}, so every lane reads only its own bytes.
-  //
-  // Block constants: lane L computes the constants of weight row
-  // warp*16kMT + (L mod 16kMT) (all four blocks when kMT = 2, blocks
-  // 2(L / 16) and 2(L / 16) + 1 when kMT = 1) and stores them in a two-slot
-  // table in the free halves of pair-table rows 0..63; the lanes that read them
-  // belong to the same warp.
-  const int g = lane >> 2, t = lane & 3;
-  const int pg = ((g & 3) << 1) | (g >> 2);
-  const uint32_t tbase = kTableAddr | (static_cast<uint32_t>(lane) << 2);
-  const uint32_t crow = static_cast<uint32_t>(warp * kRW + pg) * 128u;
-  const float mu = __ldg(a.mean);
-  const uint32_t kbl = static_cast<uint32_t>(kblocks);
-
-  const int crow_l = warp * kRW + (lane & (kRW - 1));          // this lane's constant row
-  const int cb0 = kMT == 2 ? 0 : 2 * (lane >> 4);              // its first block
-  auto cblk0 = [&](Pos p) -> uint32_t {                        // block indices < 2^32
-    return static_cast<uint32_t>(p.tile * kRows + crow_l) * kbl + 4u * p.step;
-  };
-  auto load_raw = [&](Pos p, bool valid, RowConsts& k) {
-    k.q = 0;
-    k.c2a = 0.0f;
-    k.c2b = 0.0f;
-    if (valid && p.tile * kRows + crow_l < a.nw) {
-      const uint32_t blk0 = cblk0(p);
-      if (kQuad) {
-        k.q = __ldg(reinterpret_cast<const uint32_t*>(a.qabs + blk0));
-        k.c2a = __ldg(a.c2 + (blk0 >> 8));
-      } else {
-        const int nb = min(4, kblocks - 4 * p.step);
+  if (warp >= kConsumerWarps) {
+    // ------------------------------------------------ producer warps
+    // Thread 0 of warp 8 streams the [256 rows x 128 bytes] code tile
+    // (128B-swizzled) and the four [m x 64] activation boxes of each step into
+    // the ring; producer warp h writes the step's block constants of tile rows
+    // 64 h + lane + 32 j (j < 2) into the stage's slot.  The consumers only wait
+    // for the barrier initialisation.
+    const int hw = warp - kConsumerWarps;
+    const bool tma_thread = hw == 0 && lane == 0;
+    named_barrier_sync(2, kProducerWarps * 32);   // barrier initialisation seen by all producers
+    named_barrier_arrive(1, kGemvThreads);
+    const float mu = __ldg(a.mean);
+    auto load_raw = [&](Pos p, bool valid, RowConsts (&k)[kRowsPerProducerLane]) {
+#pragma unroll
+      for (int j = 0; j < kRowsPerProducerLane; ++j) {
+        k[j].q = 0;
+        k[j].c2a = 0.0f;
+        k[j].c2b = 0.0f;
+        const int64_t row = static_cast<int64_t>(p.tile) * kRows + 64 * hw + lane + 32 * j;
+        if (valid && row < a.nw) {
+          const uint32_t blk0 = static_cast<uint32_t>(row) * kbl + 4u * static_cast<uint32_t>(p.step);
+          if (kQuad) {
+            k[j].q = __ldg(reinterpret_cast<const uint32_t*>(a.qabs + blk0));
+            k[j].c2a = __ldg(a.c2 + (blk0 >> 8));
+          } else {
+            const int nb = min(4, kblocks - 4 * p.step);
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+              if (b < nb) k[j].q |= static_cast<uint32_t>(__ldg(a.qabs + blk0 + b)) << (8 * b);
+            k[j].c2a = __ldg(a.c2 + (blk0 >> 8));
+            k[j].c2b = __ldg(a.c2 + ((blk0 + nb - 1) >> 8));
+          }
+        }
+      }
+    };
+    // c2 / 448 of the group last seen by each of the lane's rows
+    uint32_t grp_cache[kRowsPerProducerLane];
+    float c2q_cache[kRowsPerProducerLane];
+#pragma unroll
+    for (int j = 0; j < kRowsPerProducerLane; ++j) { grp_cache[j] = 0xFFFFFFFFu; c2q_cache[j] = 0.0f; }
+    // c[b] = fma(e4m3(q_b), c2 / 448, mu) for the lane's rows of step p into slot `slot`
+    auto write_consts = [&](Pos p, const RowConsts (&k)[kRowsPerProducerLane], uint32_t slot) {
+#pragma unroll
+      for (int j = 0; j < kRowsPerProducerLane; ++j) {
+        const int64_t row = static_cast<int64_t>(p.tile) * kRows + 64 * hw + lane + 32 * j;
+        const uint32_t blk0 = static_cast<uint32_t>(row) * kbl + 4u * static_cast<uint32_t>(p.step);
+        const uint32_t grp = blk0 >> 8;
+        if (grp != grp_cache[j]) {
+          grp_cache[j] = grp;
+          c2q_cache[j] = __fdiv_rn(k[j].c2a, 448.0f);
+        }
+        float f[4];
+        e4m3x4_to_f32(k[j].q, f);
+        float c[4];
+        if (kQuad) {
+#pragma unroll
+          for (int b = 0; b < 4; ++b) c[b] = __fmaf_rn(f[b], c2q_cache[j], mu);
+        } else {
+          const float c2q_b = __fdiv_rn(k[j].c2b, 448.0f);
+#pragma unroll
+          for (int b = 0; b < 4; ++b)
+            c[b] = __fmaf_rn(f[b], ((blk0 + b) >> 8) == grp ? c2q_cache[j] : c2q_b, mu);
+        }
+        const uint32_t r = static_cast<uint32_t>(64 * hw + lane + 32 * j);
+        sts128(hole(32u * slot + (r >> 3), (r & 7u) * 16u), c[0], c[1], c[2], c[3]);
+      }
+    };
+    const uint32_t xbytes = 4u * static_cast<uint32_t>(m) * 128u;
+    Pos p = first;
+    Pos p2 = advance(advance(first));
+    RowConsts ra[kRowsPerProducerLane], rb[kRowsPerProducerLane];                // raw constants of steps it and it + 1
+    load_raw(first, n_mine > 0, ra);
+    load_raw(advance(first), n_mine > 1, rb);
+    uint32_t ps = 0, pph = 0;
+    for (int64_t it = 0; it < n_mine; ++it) {
+      RowConsts rc[kRowsPerProducerLane];
+      load_raw(p2, it + 2 < n_mine, rc);  // two steps ahead
+      // stage ps is free once every consumer warp released its previous use
+      bool ok = true;
+      if (lane == 0) ok = mbar_test_wait(&empty[ps], pph ^ 1u) || mbar_wait(&empty[ps], pph ^ 1u, a.err);
+      if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
+      if (tma_thread) {
+        mbar_arrive_expect_tx(&full[ps], kCodeTile + xbytes);
+        const int col0 = p.step * kStepCols;
+        tma_load_2d(gptr(code_stage(ps)), &cmap, col0 / 2, p.tile * kRows, &full[ps]);
 #pragma unroll
         for (int b = 0; b < 4; ++b)
-          if (b < nb) k.q |= static_cast<uint32_t>(__ldg(a.qabs + blk0 + b)) << (8 * b);
-        k.c2a = __ldg(a.c2 + (blk0 >> 8));
-        k.c2b = __ldg(a.c2 + ((blk0 + nb - 1) >> 8));
+          tma_load_2d(gptr(xs0 + ps * kXTile + b * kXBox), &xmap, col0 + b * 64, 0, &full[ps]);
       }
-    }
-  };
-  uint32_t grp_cache = 0xFFFFFFFFu;
-  float c2q_cache = 0.0f;
-  // c[b] = fma(e4m3(q_b), c2 / 448, mu) for the lane's row and blocks, into slot `slot`
-  auto write_consts = [&](Pos p, const RowConsts& k, uint32_t slot) {
-    const uint32_t blk0 = cblk0(p);
-    const uint32_t grp = blk0 >> 8;
-    if (grp != grp_cache) {
-      grp_cache = grp;
-      c2q_cache = __fdiv_rn(k.c2a, 448.0f);
-    }
-    float f[4];
-    e4m3x4_to_f32(k.q, f);
-    float c[4];
-    if (kQuad) {
+      write_consts(p, ra, ps);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full[ps]);   // the warp's constant stores are ordered before it
 #pragma unroll
-      for (int b = 0; b < 4; ++b) c[b] = __fmaf_rn(f[b], c2q_cache, mu);
-    } else {
-      const float c2q_b = __fdiv_rn(k.c2b, 448.0f);
-#pragma unroll
-      for (int b = 0; b < 4; ++b) c[b] = __fmaf_rn(f[b], ((blk0 + b) >> 8) == grp ? c2q_cache : c2q_b, mu);
+      for (int j = 0; j < kRowsPerProducerLane; ++j) { ra[j] = rb[j]; rb[j] = rc[j]; }
+      p = advance(p);
+      p2 = advance(p2);
+      if (++ps == kStages) { ps = 0; pph ^= 1u; }
     }
-    const uint32_t e = slot * 256u + static_cast<uint32_t>(crow_l);
-    if (kMT == 2) {
-      sts128(hole(e >> 3, (e & 7u) * 16u), c[0], c[1], c[2], c[3]);
-    } else {
-      const float c0 = cb0 == 0 ? c[0] : c[2], c1 = cb0 == 0 ? c[1] : c[3];
-      asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(hole(e >> 3, (e & 7u) * 16u + cb0 * 4u)),
-                   "f"(c0), "f"(c1) : "memory");
-    }
-  };
-
-  Pos pos = first;
-  Pos pos1 = advance(pos), pos2 = advance(pos1), pos3 = advance(pos2);
-  RowConsts r0, ra, rb;                   // raw inputs of steps 0, it + 1 and it + 2
-  load_raw(pos, n_mine > 0, r0);
-  load_raw(pos1, n_mine > 1, ra);
-  load_raw(pos2, n_mine > 2, rb);
-
-  if (threadIdx.x < 16) s_level[threadIdx.x] = a.level[threadIdx.x];
-  __syncthreads();                        // levels, barrier initialisation
-  // the first loads are in flight while the pair table is built
-  if (producer)
-    for (int i = 0; i < kStages - 1; ++i) issue_next(true);
+    return;
+  }
   // pair table: entry (byte v, lane l) = {bf16(L[v >> 4]), bf16(L[v & 15])}, element order;
-  // thread v converts entry v once and writes its 32 copies
-  for (int v = threadIdx.x; v < 256; v += kThreads) {
-    const __nv_bfloat162 e = __floats2bfloat162_rn(s_level[v >> 4], s_level[v & 15]);
+  // consumer thread v converts entry v once and writes its 32 copies
+  {
+    const int v = threadIdx.x;
+    const __nv_bfloat162 e = __floats2bfloat162_rn(a.level[v >> 4], a.level[v & 15]);
     const float ev = __uint_as_float(*reinterpret_cast<const uint32_t*>(&e));
 #pragma unroll
     for (int l = 0; l < 32; l += 4) sts128(kTableAddr + v * 256 + l * 4, ev, ev, ev, ev);
   }
-  write_consts(pos, r0, 0);
-  __syncthreads();                        // pair table and step 0's constants in place
-  launch_dependents();                    // k_finish may be scheduled; it waits for this grid
+  named_barrier_sync(1, kGemvThreads);    // pair table written, barriers initialised
+
+  // ------------------------------------------------ consumer warps
+  // Lane (g, t) serves MMA rows g and g + 8 of the warp's two m16 tiles.  MMA
+  // row g of an 8-row group is weight row 8u + pg with pg = 2(g mod 4) + g / 4,
+  // so that the lanes of each half-warp read rows whose 128-byte swizzle
+  // patterns differ in bits 1 and 2 (no bank conflicts).  The lane's rows are
+  // warp*32 + 8q + pg (q < 4; tile i uses q = 2i and 2i + 1).  In every
+  // 64-column block the lane reads the code bytes [8t, 8t + 8) of those rows.
+  // Columns enter the MMA in a permuted order (the same for X): slice j of a
+  // block feeds columns 16t + 4j + {0, 1} as k = {2t, 2t+1} and 16t + 4j + {2, 3}
+  // as k = {2t+8, 2t+9}, so every lane reads only its own bytes.  The LoRA
+  // up-projection uses the same order over each 64-column group of the rank.
+  const int g = lane >> 2, t = lane & 3;
+  const int pg = ((g & 3) << 1) | (g >> 2);
+  const uint32_t tbase = kTableAddr | (static_cast<uint32_t>(lane) << 2);
+  const uint32_t crow = static_cast<uint32_t>(warp * 32 + pg) * 128u;
 
   // X rows of this lane (token 8n + g); lanes of tokens >= m load nothing, and
   // the MMA columns they feed are never stored.
@@ -361,56 +379,194 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
     for (int jp = 0; jp < 2; ++jp) xoff[n][jp] = (8 * n + g) * 128 + ((((2u * t) + jp) ^ g) << 4);
   }
 
-  float y[kMT][kNT][4];
+  // s X A^T as bf16 [token][64 lora_steps]: 16-byte chunk c of token i's
+  // 64-column group q sits in hole row kSxaHole + i lora_steps + q at chunk
+  // c ^ (i mod 8), so that the eight tokens read by a quarter-warp hit
+  // different banks.
+  auto sxa_addr = [&](int tok, int grp, int chunk) -> uint32_t {
+    return hole(kSxaHole + static_cast<uint32_t>(tok * a.lora_steps + grp),
+                static_cast<uint32_t>((chunk ^ (tok & 7)) << 4));
+  };
+  // Sum k_xa_zero's K slices of X A^T (the consumer threads share the chunks of
+  // eight columns), write X A^T out from CTA 0 when asked, stage bf16(s X A^T).
+  auto stage_sxa = [&]() {
+    const int c8n = a.lora_steps * 8;               // 8-column chunks per token
+    const int nchunk = m * c8n;
+    for (int e = static_cast<int>(threadIdx.x); e < nchunk; e += kConsumers) {
+      const int tok = e / c8n, c8 = e - (e / c8n) * c8n;
+      const int col = 8 * c8;
+      float v[8];
 #pragma unroll
-  for (int i = 0; i < kMT; ++i)
+      for (int q = 0; q < 8; ++q) v[q] = 0.0f;
+      if (col < a.r) {                              // r is a multiple of 8
+        for (int sp = 0; sp < a.xa_splits; ++sp) {
+          const float4* src =
+              reinterpret_cast<const float4*>(a.xa_part + (static_cast<int64_t>(sp) * 16 + tok) * a.ld_xa + col);
+          const float4 u0 = __ldcg(src), u1 = __ldcg(src + 1);
+          v[0] += u0.x; v[1] += u0.y; v[2] += u0.z; v[3] += u0.w;
+          v[4] += u1.x; v[5] += u1.y; v[6] += u1.z; v[7] += u1.w;
+        }
+        if (a.xa_out && blockIdx.x == 0)
 #pragma unroll
-    for (int n = 0; n < kNT; ++n)
+          for (int q = 0; q < 8; ++q) a.xa_out[static_cast<int64_t>(tok) * a.r + col + q] = v[q];
+      }
+      uint32_t w[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) y[i][n][e] = 0.0f;
-  // The partial of the first tile this CTA touches is kept in registers until
-  // the next tile boundary (or the end of the range): by then the previous
-  // kernel (X A^T and the zeroed split buffer) has surely finished, so the wait
-  // for it does not stall the stream.
-  float ys[kMT][kNT][4];
-  int ys_tile = -1;
-  bool dep_done = false;
-  // add a tile partial to the split buffer (fire-and-forget reductions)
-  auto flush = [&](int tile, float (&v)[kMT][kNT][4]) {
+      for (int q = 0; q < 4; ++q) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(a.s, v[2 * q]), __fmul_rn(a.s, v[2 * q + 1]));
+        w[q] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sxa_addr(tok, c8 >> 3, c8 & 7)),
+                   "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
+    }
+  };
+  // Y rows of tile `tile` for this lane from its fp32 sums: add the LoRA
+  // up-projection s (X A^T) B^T with warp MMAs (A operand = rows of B, B operand
+  // = the staged bf16(s X A^T)) and store bf16.
+  auto finish = [&](int tile, float (&acc)[2][kNT][4]) {
+    const int64_t row0 = static_cast<int64_t>(tile) * kRows + warp * 32 + pg;
+    for (int grp = 0; grp < a.lora_steps; ++grp) {
+      uint4 xs[kNT][2];
 #pragma unroll
-    for (int i = 0; i < kMT; ++i)
+      for (int n = 0; n < kNT; ++n)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint4 u;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w)
+                       : "r"(sxa_addr(8 * n + g, grp, 2 * t + hf)) : "memory");
+          xs[n][hf] = u;
+        }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        uint4 bv[2][2];                             // [row half][8-column half]
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const int64_t row = row0 + 8 * (2 * i + h);
+            const int col = grp * 64 + 16 * t + 8 * hf;
+            bv[h][hf] = (row < a.nw && col < a.r)
+                            ? __ldg(reinterpret_cast<const uint4*>(a.lora_b + row * a.r + col))
+                            : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            const uint32_t a0 = kk ? bv[0][hf].z : bv[0][hf].x, a1 = kk ? bv[1][hf].z : bv[1][hf].x;
+            const uint32_t a2 = kk ? bv[0][hf].w : bv[0][hf].y, a3 = kk ? bv[1][hf].w : bv[1][hf].y;
+#pragma unroll
+            for (int n = 0; n < kNT; ++n) {
+              const uint32_t b0 = kk ? xs[n][hf].z : xs[n][hf].x, b1 = kk ? xs[n][hf].w : xs[n][hf].y;
+              mma_bf16_16816(acc[i][n], a0, a1, a2, a3, b0, b1);
+            }
+          }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
 #pragma unroll
       for (int n = 0; n < kNT; ++n)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int64_t row = static_cast<int64_t>(tile) * kRows + warp * kRW + 8 * (2 * i + (e >> 1)) + pg;
+          const int64_t row = row0 + 8 * (2 * i + (e >> 1));
           const int tok = 8 * n + 2 * t + (e & 1);
-          if (row < a.nw && tok < m) atomicAdd(a.yacc + tok * a.nw + row, v[i][n][e]);
+          if (row < a.nw && tok < m) {
+            const __nv_bfloat16 h = __float2bfloat16_rn(acc[i][n][e]);
+            a.y[tok * a.nw + row] = *reinterpret_cast<const uint16_t*>(&h);
+          }
         }
   };
+  // Tile partials.  A CTA's share touches at most two tiles that other CTAs
+  // share too, its first and its last; every tile inside the share lies in
+  // it alone.  At the end of its part of a tile a warp writes its fp32 partial
+  // to one of the CTA's two slots (plain stores, [cta][2][warp][lane][16]
+  // floats) and counts itself in the tile's per-warp counter; the warp whose
+  // arrival completes the count sums the slots of every CTA of the tile and
+  // finishes those 32 rows.
+  auto shares_of = [&](int tile) -> int {
+    const int64_t u0 = static_cast<int64_t>(tile) * steps;
+    return static_cast<int>(owner_of(u0 + steps - 1, total, ctas) - owner_of(u0, total, ctas) + 1);
+  };
+  auto slot_ptr = [&](int64_t cta, int sl) -> float4* {
+    return reinterpret_cast<float4*>(a.slots + (((cta * 2 + sl) * kConsumerWarps + warp) * 32 + lane) * 16);
+  };
+  auto put_slot = [&](int sl, const float (&v)[2][kNT][4]) {
+    float4* d = slot_ptr(blockIdx.x, sl);
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int n = 0; n < kNT; ++n) d[i * kNT + n] = make_float4(v[i][n][0], v[i][n][1], v[i][n][2], v[i][n][3]);
+  };
+  // count this warp's partial of `tile` (already in its slot); the last one
+  // finishes the tile, with `v` as scratch
+  auto arrive = [&](int tile, float (&v)[2][kNT][4]) {
+    const int shares = shares_of(tile);
+    __threadfence();
+    __syncwarp();
+    uint32_t before = 0;
+    if (lane == 0) before = atomicAdd(a.cnt + static_cast<int64_t>(tile) * kConsumerWarps + warp, 1u);
+    before = __shfl_sync(0xFFFFFFFFu, before, 0);
+    if (static_cast<int>(before) + 1 != shares) return;
+    __threadfence();
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int n = 0; n < kNT; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[i][n][e] = 0.0f;
+    const int64_t u0 = static_cast<int64_t>(tile) * steps;
+    const int64_t c0 = owner_of(u0, total, ctas);
+    for (int64_t c = c0; c < c0 + shares; ++c) {
+      // the tile is CTA c's first tile unless c's share starts before it
+      const int sl = bound(static_cast<int>(c), total, ctas) >= u0 ? 0 : 1;
+      const float4* src = slot_ptr(c, sl);
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int n = 0; n < kNT; ++n) {
+          const float4 q = __ldcg(src + i * kNT + n);
+          v[i][n][0] += q.x; v[i][n][1] += q.y; v[i][n][2] += q.z; v[i][n][3] += q.w;
+        }
+    }
+    finish(tile, v);
+  };
 
+  float y[2][kNT][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int n = 0; n < kNT; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) y[i][n][e] = 0.0f;
+  // The first tile's partial goes to slot 0 at once; its count waits for the
+  // next tile boundary (or the end of the share), when the previous kernel
+  // (X A^T slices, zeroed counters) has surely finished, so the wait for it
+  // does not stall the stream.
+  int pending = -1;
+  bool dep_done = false;
+
+  Pos pos = first;
   uint32_t s = 0, ph = 0;
   bool alive = true;
-  for (int64_t it = 0; it < n_mine && alive; ++it) {
-    // this step's constants c[q][b] for the lane's rows warp*16kMT + 8q + pg
-    float c[2 * kMT][4];
-    const uint32_t cslot = static_cast<uint32_t>(it & 1) * 256u;
+  for (int64_t it = 0; it < n_mine; ++it) {
+    // the stage of this step: test first (cheap when the data is already there)
+    if (!mbar_test_wait(&full[s], ph) && !mbar_wait(&full[s], ph, a.err)) { alive = false; break; }
+    // this step's constants c[q][b] for the lane's rows warp*32 + 8q + pg
+    float c[4][4];
 #pragma unroll
-    for (int q = 0; q < 2 * kMT; ++q) {
-      const uint32_t e = cslot + static_cast<uint32_t>(warp * kRW + 8 * q + pg);
-      const float4 v = lds128f(hole(e >> 3, (e & 7u) * 16u));
+    for (int q = 0; q < 4; ++q) {
+      const float4 v = lds128f(hole(32u * s + 4u * warp + q, static_cast<uint32_t>(pg) * 16u));
       c[q][0] = v.x; c[q][1] = v.y; c[q][2] = v.z; c[q][3] = v.w;
     }
-    // the stage of this step: test first (cheap when the data is already there)
-    if (!mbar_test_wait(&full[s], ph) && !mbar_wait(&full[s], ph, a.err)) break;
     const uint32_t cs = code_stage(s) + crow;
     const uint32_t xs = xs0 + s * kXTile;
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
       const uint32_t coff = ((((2u * b) + (t >> 1)) ^ pg) << 4) | ((t & 1u) << 3);
-      uint2 cw[2 * kMT];
+      uint2 cw[4];
 #pragma unroll
-      for (int q = 0; q < 2 * kMT; ++q) cw[q] = lds64(cs + q * 1024u + coff);
+      for (int q = 0; q < 4; ++q) cw[q] = lds64(cs + q * 1024u + coff);
       uint4 xv[kNT][2];
 #pragma unroll
       for (int n = 0; n < kNT; ++n)
@@ -420,20 +576,13 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);                // stage fully read
       }
-      if (b == 1) {
-        // next step's constants into the other slot (read two steps ago by
-        // this warp; the syncwarp at b == 3 orders them before their readers)
-        __syncwarp();
-        if (it + 1 < n_mine) write_consts(pos1, ra, static_cast<uint32_t>((it + 1) & 1));
-      }
-      if (producer && !issue_next(b == 3)) { alive = false; break; }
-      float p[kMT][kNT][4];                                   // [m tile][n tile][element]
+      float p[2][kNT][4];                                     // [m tile][n tile][element]
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const uint32_t sel0 = 0x7604u | ((2u * (j & 1)) << 4);   // byte 2(j&1) of the word
         const uint32_t sel1 = sel0 + 0x10u;                      // byte 2(j&1) + 1
 #pragma unroll
-        for (int i = 0; i < kMT; ++i) {
+        for (int i = 0; i < 2; ++i) {
           const uint32_t w0 = (j < 2) ? cw[2 * i].x : cw[2 * i].y;
           const uint32_t w1 = (j < 2) ? cw[2 * i + 1].x : cw[2 * i + 1].y;
           const uint32_t a0 = lds_table(__byte_perm(w0, tbase, sel0));
@@ -450,61 +599,46 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
         }
       }
 #pragma unroll
-      for (int i = 0; i < kMT; ++i)
+      for (int i = 0; i < 2; ++i)
 #pragma unroll
         for (int n = 0; n < kNT; ++n)
 #pragma unroll
           for (int e = 0; e < 4; ++e) y[i][n][e] = __fmaf_rn(c[2 * i + (e >> 1)][b], p[i][n][e], y[i][n][e]);
     }
-    if (!alive) break;
 
     if (pos.step == steps - 1 || it == n_mine - 1) {
-      // end of this CTA's share of the tile
-      if (!dep_done && ys_tile < 0 && it != n_mine - 1) {
-        ys_tile = pos.tile;                                   // keep it for later
-#pragma unroll
-        for (int i = 0; i < kMT; ++i)
-#pragma unroll
-          for (int n = 0; n < kNT; ++n)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) ys[i][n][e] = y[i][n][e];
+      // end of this CTA's share of the tile: its partial goes to the slot (0 for
+      // the share's first tile, else 1; a tile inside the share is counted and
+      // finished at once, so slot 1 is free again for the next one)
+      put_slot(pos.tile == first.tile ? 0 : 1, y);
+      if (!dep_done && pending < 0 && it != n_mine - 1) {
+        pending = pos.tile;                                   // counted later
       } else {
         if (!dep_done) {
           grid_dependency_wait();
           dep_done = true;
+          stage_sxa();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(xa_bar);
+          if (!mbar_test_wait(xa_bar, 0) && !mbar_wait(xa_bar, 0, a.err)) { alive = false; break; }
         }
-        if (ys_tile >= 0) {
-          flush(ys_tile, ys);
-          ys_tile = -1;
+        for (int k = 0; k < 2; ++k) {
+          const int tl = k == 0 ? pending : pos.tile;
+          if (tl >= 0) arrive(tl, y);
         }
-        flush(pos.tile, y);
+        pending = -1;
       }
 #pragma unroll
-      for (int i = 0; i < kMT; ++i)
+      for (int i = 0; i < 2; ++i)
 #pragma unroll
         for (int n = 0; n < kNT; ++n)
 #pragma unroll
           for (int e = 0; e < 4; ++e) y[i][n][e] = 0.0f;
     }
-    ra = rb;                                   // loaded a full step ago
-    load_raw(pos3, it + 3 < n_mine, rb);
-    pos = pos1; pos1 = pos2; pos2 = pos3; pos3 = advance(pos3);
+    pos = advance(pos);
     if (++s == kStages) { s = 0; ph ^= 1u; }
   }
-  if (!alive) return;
-  // this CTA's share of X A^T: the sum of k_xa_zero's K slices (complete once
-  // the wait above has returned; every CTA reached it at its last flush)
-  {
-    const int nxa = m * a.r;
-    const int e_beg = static_cast<int>((static_cast<int64_t>(nxa) * blockIdx.x) / gridDim.x);
-    const int e_end = static_cast<int>((static_cast<int64_t>(nxa) * (blockIdx.x + 1)) / gridDim.x);
-    for (int e = e_beg + static_cast<int>(threadIdx.x); e < e_end; e += kThreads) {
-      const int i = e / a.r, j = e - (e / a.r) * a.r;
-      float v = 0.0f;
-      for (int sp = 0; sp < a.xa_splits; ++sp) v += __ldcg(a.xa_part + (static_cast<int64_t>(sp) * 16 + i) * a.ld_xa + j);
-      a.xa[i * a.ld_xa + j] = v;
-    }
-  }
+  (void)alive;
 }
 
 // Partial X A^T and the zeroed split buffer of k_gemv.  CTA (c, sp) computes
@@ -583,98 +717,6 @@ k_xa_zero(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A, int64_
   for (int64_t e = gtid; e < n4; e += nthreads) zero4[e] = z;
 }
 
-// Y[i, n] = bf16(split[i, n] + s * sum_c XA[i, c] B[n, c]).  Four lanes per
-// row n: lane q of the four takes the 8-column chunks cc = q, q + 4, ... of the
-// rank, the four partial sums are combined with two butterfly shuffles, and
-// lane q stores the tokens i = q, q + 4, ...  kMaxM (1, 4, 8 or 16) bounds the
-// token count at compile time.
-template <int kMaxM>
-__global__ void __launch_bounds__(128)
-k_finish(const float* __restrict__ yacc, const float* __restrict__ xa, int64_t ld_xa,
-         const uint16_t* __restrict__ lora_b, int r, float s, int64_t m, int64_t nw, uint16_t* __restrict__ y,
-         float* __restrict__ xa_out) {
-  __shared__ __align__(16) float s_xa[kMaxM * 256];
-  grid_dependency_wait();                  // k_gemv complete (it waited for k_xa_zero)
-  const int mi = static_cast<int>(m);
-  // X A^T into shared memory (row i at i * r)
-  for (int j = threadIdx.x; j < r; j += blockDim.x) {
-    float v[kMaxM];
-#pragma unroll
-    for (int i = 0; i < kMaxM; ++i) v[i] = i < mi ? __ldcg(xa + i * ld_xa + j) : 0.0f;
-#pragma unroll
-    for (int i = 0; i < kMaxM; ++i)
-      if (i < mi) {
-        s_xa[i * r + j] = v[i];
-        if (xa_out && blockIdx.x == 0) xa_out[i * r + j] = v[i];
-      }
-  }
-  const int q = threadIdx.x & 3;
-  const int64_t n = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 4) + (threadIdx.x >> 2);
-  const bool live = n < nw;                // all lanes stay for the shuffles
-  // split-buffer values of this lane's tokens and its first B chunks are issued
-  // before the barrier, with the staging loads: one memory round trip per row
-  constexpr int kMine = (kMaxM + 3) / 4;   // tokens stored by this lane
-  float acc[kMine];
-#pragma unroll
-  for (int u = 0; u < kMine; ++u) {
-    const int i = q + 4 * u;
-    acc[u] = (live && i < mi) ? __ldcg(yacc + i * nw + n) : 0.0f;
-  }
-  const uint4* brow = reinterpret_cast<const uint4*>(lora_b + (live ? n : 0) * r);
-  const int nch = r / 8;
-  uint4 bv[4];
-#pragma unroll
-  for (int u = 0; u < 4; ++u) bv[u] = (live && q + 4 * u < nch) ? __ldg(brow + q + 4 * u) : make_uint4(0u, 0u, 0u, 0u);
-  __syncthreads();                         // X A^T staged
-  float lo[kMaxM];
-#pragma unroll
-  for (int i = 0; i < kMaxM; ++i) lo[i] = 0.0f;
-  for (int c0 = q; c0 < nch; c0 += 16) {   // four chunks of eight rank columns per round
-    if (c0 != q) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        bv[u] = (live && c0 + 4 * u < nch) ? __ldg(brow + c0 + 4 * u) : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int cc = c0 + 4 * u;
-      if (cc >= nch) break;
-      const float b8[8] = {bf16_lo(bv[u].x), bf16_hi(bv[u].x), bf16_lo(bv[u].y), bf16_hi(bv[u].y),
-                           bf16_lo(bv[u].z), bf16_hi(bv[u].z), bf16_lo(bv[u].w), bf16_hi(bv[u].w)};
-#pragma unroll
-      for (int i = 0; i < kMaxM; ++i)
-        if (i < mi) {
-          const float4 x0 = *reinterpret_cast<const float4*>(&s_xa[i * r + cc * 8]);
-          const float4 x1 = *reinterpret_cast<const float4*>(&s_xa[i * r + cc * 8 + 4]);
-          float v = lo[i];
-          v = __fmaf_rn(x0.x, b8[0], v); v = __fmaf_rn(x0.y, b8[1], v);
-          v = __fmaf_rn(x0.z, b8[2], v); v = __fmaf_rn(x0.w, b8[3], v);
-          v = __fmaf_rn(x1.x, b8[4], v); v = __fmaf_rn(x1.y, b8[5], v);
-          v = __fmaf_rn(x1.z, b8[6], v); v = __fmaf_rn(x1.w, b8[7], v);
-          lo[i] = v;
-        }
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < kMaxM; ++i) {
-    lo[i] += __shfl_xor_sync(0xFFFFFFFFu, lo[i], 1);
-    lo[i] += __shfl_xor_sync(0xFFFFFFFFu, lo[i], 2);
-  }
-  if (!live) return;
-#pragma unroll
-  for (int u = 0; u < kMine; ++u) {
-    const int i = q + 4 * u;
-    float v = lo[0];                         // lo[i] with compile-time indices
-#pragma unroll
-    for (int k = 1; k < kMaxM; ++k)
-      if (k == i) v = lo[k];
-    if (i < mi) {
-      const __nv_bfloat16 h = __float2bfloat16_rn(__fmaf_rn(s, v, acc[u]));
-      y[i * nw + n] = *reinterpret_cast<const uint16_t*>(&h);
-    }
-  }
-}
-
 cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, void** args) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
@@ -686,10 +728,12 @@ cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaS
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelExC(&cfg, fn, args);
+  const cudaError_t e = cudaLaunchKernelExC(&cfg, fn, args);
+  if (e != cudaSuccess) (void)cudaGetLastError();   // leave no stale error for the next launch check
+  return e;
 }
 
-template <int kNT, bool kQuad, int kMT>
+template <int kNT, bool kQuad>
 cudaError_t launch_gemv_t(const GemvArgs& args, const CUtensorMap& cm, const CUtensorMap& xm, int num_sms,
                           cudaStream_t stream) {
   static std::atomic<uint64_t> attr_done{0};
@@ -698,35 +742,33 @@ cudaError_t launch_gemv_t(const GemvArgs& args, const CUtensorMap& cm, const CUt
   if (e != cudaSuccess) return e;
   const uint64_t bit = 1ull << (dev & 63);
   if (!(attr_done.load(std::memory_order_acquire) & bit)) {
-    e = cudaFuncSetAttribute(k_gemv<kNT, kQuad, kMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(k_gemv<kNT, kQuad>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(GemvStages<kNT>::kSmemTop));
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(bit, std::memory_order_acq_rel);
   }
+  // no more CTAs than steps, so that every CTA's share is non-empty
   const int64_t total = static_cast<int64_t>(args.m_tiles) * args.steps;
-  const unsigned grid = static_cast<unsigned>(total < num_sms ? total : num_sms);
+  int64_t grid64 = total < num_sms ? total : num_sms;
+  if (grid64 > kMaxGemvCtas) grid64 = kMaxGemvCtas;
+  const unsigned grid = static_cast<unsigned>(grid64);
   GemvArgs a = args;
   CUtensorMap c = cm, x = xm;
   void* kargs[3] = {&a, &c, &x};
   // dynamic shared memory up to the map's top covers any start address of the window
-  return launch_pdl(reinterpret_cast<const void*>(k_gemv<kNT, kQuad, kMT>), dim3(grid),
-                    dim3(GemvShape<kMT>::kThreads), GemvStages<kNT>::kSmemTop, stream, kargs);
-}
-
-template <int kMT>
-cudaError_t launch_gemv_mt(const GemvArgs& args, const CUtensorMap& cm, const CUtensorMap& xm, int num_sms,
-                           cudaStream_t stream) {
-  const bool quad = (args.kw / 64) % 4 == 0;
-  if (args.m <= 8)
-    return quad ? launch_gemv_t<1, true, kMT>(args, cm, xm, num_sms, stream)
-                : launch_gemv_t<1, false, kMT>(args, cm, xm, num_sms, stream);
-  return quad ? launch_gemv_t<2, true, kMT>(args, cm, xm, num_sms, stream)
-              : launch_gemv_t<2, false, kMT>(args, cm, xm, num_sms, stream);
+  return launch_pdl(reinterpret_cast<const void*>(k_gemv<kNT, kQuad>), dim3(grid), dim3(kGemvThreads),
+                    GemvStages<kNT>::kSmemTop, stream, kargs);
 }
 
 }  // namespace
 
 int gemv_tile_rows() { return kRows; }
+
+int64_t gemv_slot_floats(int64_t m_tiles, int64_t steps) {
+  int64_t ctas = m_tiles * steps;
+  if (ctas > kMaxGemvCtas) ctas = kMaxGemvCtas;
+  return ctas * 2 * kConsumerWarps * 32 * 16;
+}
 
 cudaError_t launch_xa_zero(const uint16_t* X, const uint16_t* A, int64_t m, int64_t kw, int r, float* part,
                            int64_t ld, int splits, float* zero, int64_t n_zero, cudaStream_t stream) {
@@ -751,22 +793,12 @@ int xa_splits_for(int r, int64_t kw) {
 
 cudaError_t launch_gemv(const GemvArgs& args, const CUtensorMap& codes_map, const CUtensorMap& x_map,
                         int num_sms, cudaStream_t stream) {
-#ifdef GEMV_FORCE_MT
-  return launch_gemv_mt<GEMV_FORCE_MT>(args, codes_map, x_map, num_sms, stream);
-#else
-  return launch_gemv_mt<2>(args, codes_map, x_map, num_sms, stream);
-#endif
-}
-
-cudaError_t launch_gemv_finish(const float* yacc, const float* xa, int64_t ld_xa, const uint16_t* lora_b, int r,
-                               float s, int64_t m, int64_t nw, uint16_t* y, float* xa_out, cudaStream_t stream) {
-  void* kargs[10] = {&yacc, &xa, &ld_xa, &lora_b, &r, &s, &m, &nw, &y, &xa_out};
-  const unsigned grid = static_cast<unsigned>((nw + 31) / 32);      // 32 rows per 128-thread CTA
-  const void* fn = m <= 1 ? reinterpret_cast<const void*>(k_finish<1>)
-                 : m <= 4 ? reinterpret_cast<const void*>(k_finish<4>)
-                 : m <= 8 ? reinterpret_cast<const void*>(k_finish<8>)
-                          : reinterpret_cast<const void*>(k_finish<16>);
-  return launch_pdl(fn, dim3(grid), dim3(128), 0, stream, kargs);
+  const bool quad = (args.kw / 64) % 4 == 0;
+  if (args.m <= 8)
+    return quad ? launch_gemv_t<1, true>(args, codes_map, x_map, num_sms, stream)
+                : launch_gemv_t<1, false>(args, codes_map, x_map, num_sms, stream);
+  return quad ? launch_gemv_t<2, true>(args, codes_map, x_map, num_sms, stream)
+              : launch_gemv_t<2, false>(args, codes_map, x_map, num_sms, stream);
 }
 
 }  // namespace qlora

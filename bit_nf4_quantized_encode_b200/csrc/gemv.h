@@ -13,12 +13,17 @@ struct GemvArgs {
   const float* mean;         // per-tensor mean
   int64_t nw, kw;            // W shape (rows = out features, cols = in features)
   int64_t m;                 // token rows (<= 16)
-  float* yacc;               // fp32 [m, nw] accumulator, zeroed by k_xa_zero
+  float* slots;              // fp32 [gemv_slot_floats()] partials of shared tiles
+  uint32_t* cnt;             // [m_tiles * 8] per-warp tile counters, zeroed by k_xa_zero
   const float* xa_part;      // k_xa_zero's X A^T slices: [xa_splits][16][ld_xa] fp32
-  float* xa;                 // X A^T [m, ld_xa] fp32, summed by k_gemv at its end
-  int64_t ld_xa;
-  int r;                     // LoRA rank
+  int64_t ld_xa;             // 64 lora_steps
+  int r;                     // LoRA rank (a multiple of 8)
+  int lora_steps;            // 64-column groups of the rank
   int xa_splits;
+  float s;                   // LoRA scale alpha / r
+  const uint16_t* lora_b;    // B bf16 [nw, r]
+  uint16_t* y;               // Y bf16 [m, nw]
+  float* xa_out;             // X A^T fp32 [m, r], or null
   int m_tiles;               // tiles of gemv_tile_rows() weight rows
   int steps;                 // 256-column steps per row
   float level[16];           // NF4 levels
@@ -26,26 +31,25 @@ struct GemvArgs {
 };
 
 int gemv_tile_rows();
+// At most this many k_gemv CTAs (one per SM on a B200).
+constexpr int kMaxGemvCtas = 256;
+// fp32 floats of k_gemv's partial slots for a weight of m_tiles x steps units.
+int64_t gemv_slot_floats(int64_t m_tiles, int64_t steps);
 
 // Upper bound on the K slices of X A^T (the work buffer holds that many).
 constexpr int kMaxXaSplits = 16;
 // K slices of X A^T for rank r and contraction kw (1 .. kMaxXaSplits).
 int xa_splits_for(int r, int64_t kw);
 // Partial X A^T (fp32 [splits][16][ld]) for m <= 16 tokens, and the zeroing of
-// zero[n_zero] (k_gemv's split buffer; n_zero a multiple of 4, 16-byte aligned).
+// zero[n_zero] (k_gemv's tile counters; n_zero a multiple of 4, 16-byte aligned).
 cudaError_t launch_xa_zero(const uint16_t* X, const uint16_t* A, int64_t m, int64_t kw, int r, float* part,
                            int64_t ld, int splits, float* zero, int64_t n_zero, cudaStream_t stream);
 
 // codes_map: packed codes as uint8 [nw, kw/2], box {128, 256}, 128-byte swizzle.
 // x_map: X bf16 [m, kw], box {64, m}, 128-byte swizzle.
 // k_gemv is launched as a programmatic dependent of the kernel before it in the
-// stream, which must be k_xa_zero of the same call.
+// stream, which must be k_xa_zero of the same call; it writes Y (and X A^T).
 cudaError_t launch_gemv(const GemvArgs& args, const CUtensorMap& codes_map, const CUtensorMap& x_map,
                         int num_sms, cudaStream_t stream);
-
-// Y = bf16(yacc + s (X A^T) B^T), and X A^T into xa_out [m, r] when not null;
-// launched as the programmatic dependent of k_gemv.
-cudaError_t launch_gemv_finish(const float* yacc, const float* xa, int64_t ld_xa, const uint16_t* lora_b, int r,
-                               float s, int64_t m, int64_t nw, uint16_t* y, float* xa_out, cudaStream_t stream);
 
 }  // namespace qlora
