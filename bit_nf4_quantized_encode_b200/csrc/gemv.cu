@@ -142,6 +142,11 @@ __device__ __forceinline__ void named_barrier_arrive(int id, int count) {
 __device__ __forceinline__ void named_barrier_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+__device__ __forceinline__ uint32_t atomic_add_acq_rel(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
 __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
@@ -387,37 +392,47 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
     return hole(kSxaHole + static_cast<uint32_t>(tok * a.lora_steps + grp),
                 static_cast<uint32_t>((chunk ^ (tok & 7)) << 4));
   };
-  // Sum k_xa_zero's K slices of X A^T (the consumer threads share the chunks of
-  // eight columns), write X A^T out from CTA 0 when asked, stage bf16(s X A^T).
+  // Sum k_xa_zero's K slices of X A^T, write X A^T out from CTA 0 when asked,
+  // and stage bf16(s X A^T).  One lane per (8-column chunk, slice): the slices
+  // of a chunk sit in 2^sb adjacent lanes and are added by a butterfly of
+  // shuffles, so a round costs one load latency whatever the slice count.
   auto stage_sxa = [&]() {
     const int c8n = a.lora_steps * 8;               // 8-column chunks per token
     const int nchunk = m * c8n;
-    for (int e = static_cast<int>(threadIdx.x); e < nchunk; e += kConsumers) {
+    int sb = 0;
+    while ((1 << sb) < a.xa_splits) ++sb;           // at most 4 (16 slices)
+    const int sp = static_cast<int>(threadIdx.x) & ((1 << sb) - 1);
+    for (int e0 = 0; e0 < nchunk; e0 += kConsumers >> sb) {
+      const int e = e0 + (static_cast<int>(threadIdx.x) >> sb);
       const int tok = e / c8n, c8 = e - (e / c8n) * c8n;
       const int col = 8 * c8;
+      const bool live = e < nchunk && col < a.r;    // r is a multiple of 8
       float v[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) v[q] = 0.0f;
-      if (col < a.r) {                              // r is a multiple of 8
-        for (int sp = 0; sp < a.xa_splits; ++sp) {
-          const float4* src =
-              reinterpret_cast<const float4*>(a.xa_part + (static_cast<int64_t>(sp) * 16 + tok) * a.ld_xa + col);
-          const float4 u0 = __ldcg(src), u1 = __ldcg(src + 1);
-          v[0] += u0.x; v[1] += u0.y; v[2] += u0.z; v[3] += u0.w;
-          v[4] += u1.x; v[5] += u1.y; v[6] += u1.z; v[7] += u1.w;
-        }
-        if (a.xa_out && blockIdx.x == 0)
+      if (live && sp < a.xa_splits) {
+        const float4* src =
+            reinterpret_cast<const float4*>(a.xa_part + (static_cast<int64_t>(sp) * 16 + tok) * a.ld_xa + col);
+        const float4 u0 = __ldcg(src), u1 = __ldcg(src + 1);
+        v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
+        v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
+      }
+      for (int o = 1; o < (1 << sb); o <<= 1)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] += __shfl_xor_sync(0xFFFFFFFFu, v[q], o);
+      if (sp == 0 && e < nchunk) {
+        if (live && a.xa_out && blockIdx.x == 0)
 #pragma unroll
           for (int q = 0; q < 8; ++q) a.xa_out[static_cast<int64_t>(tok) * a.r + col + q] = v[q];
-      }
-      uint32_t w[4];
+        uint32_t w[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(a.s, v[2 * q]), __fmul_rn(a.s, v[2 * q + 1]));
-        w[q] = *reinterpret_cast<const uint32_t*>(&h);
+        for (int q = 0; q < 4; ++q) {
+          const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(a.s, v[2 * q]), __fmul_rn(a.s, v[2 * q + 1]));
+          w[q] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sxa_addr(tok, c8 >> 3, c8 & 7)),
+                     "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
       }
-      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sxa_addr(tok, c8 >> 3, c8 & 7)),
-                   "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
     }
   };
   // Y rows of tile `tile` for this lane from its fp32 sums: add the LoRA
@@ -502,13 +517,15 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
   // finishes the tile, with `v` as scratch
   auto arrive = [&](int tile, float (&v)[2][kNT][4]) {
     const int shares = shares_of(tile);
-    __threadfence();
+    // release: the warp's slot stores are ordered before lane 0's count (warp
+    // barrier, then a release atomic); acquire: the last warp sees every slot
+    // stored before the counts it read
     __syncwarp();
     uint32_t before = 0;
-    if (lane == 0) before = atomicAdd(a.cnt + static_cast<int64_t>(tile) * kConsumerWarps + warp, 1u);
+    if (lane == 0) before = atomic_add_acq_rel(a.cnt + static_cast<int64_t>(tile) * kConsumerWarps + warp, 1u);
     before = __shfl_sync(0xFFFFFFFFu, before, 0);
     if (static_cast<int>(before) + 1 != shares) return;
-    __threadfence();
+    __syncwarp();
 #pragma unroll
     for (int i = 0; i < 2; ++i)
 #pragma unroll
@@ -517,19 +534,41 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
         for (int e = 0; e < 4; ++e) v[i][n][e] = 0.0f;
     const int64_t u0 = static_cast<int64_t>(tile) * steps;
     const int64_t c0 = owner_of(u0, total, ctas);
-    for (int64_t c = c0; c < c0 + shares; ++c) {
-      // the tile is CTA c's first tile unless c's share starts before it
-      const int sl = bound(static_cast<int>(c), total, ctas) >= u0 ? 0 : 1;
-      const float4* src = slot_ptr(c, sl);
+    // slots in CTA order, kBatch of them in flight at a time (one for 16 tokens,
+    // whose step loop leaves no registers to spare)
+    constexpr int kBatch = kNT == 1 ? 4 : 1;
+    for (int k0 = 0; k0 < shares; k0 += kBatch) {
+      float4 q[kBatch][2 * kNT];
 #pragma unroll
-      for (int i = 0; i < 2; ++i)
+      for (int k = 0; k < kBatch; ++k)
+        if (k0 + k < shares) {
+          const int64_t c = c0 + k0 + k;
+          // the tile is CTA c's first tile unless c's share starts before it
+          const float4* src = slot_ptr(c, bound(static_cast<int>(c), total, ctas) >= u0 ? 0 : 1);
 #pragma unroll
-        for (int n = 0; n < kNT; ++n) {
-          const float4 q = __ldcg(src + i * kNT + n);
-          v[i][n][0] += q.x; v[i][n][1] += q.y; v[i][n][2] += q.z; v[i][n][3] += q.w;
+          for (int f = 0; f < 2 * kNT; ++f) q[k][f] = __ldcg(src + f);
+        }
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k)
+        if (k0 + k < shares) {
+#pragma unroll
+          for (int i = 0; i < 2; ++i)
+#pragma unroll
+            for (int n = 0; n < kNT; ++n) {
+              const float4 w = q[k][i * kNT + n];
+              v[i][n][0] += w.x; v[i][n][1] += w.y; v[i][n][2] += w.z; v[i][n][3] += w.w;
+            }
         }
     }
     finish(tile, v);
+  };
+  // LoRA B rows of a tile into L2 ahead of its finish (lane (g, t) takes row
+  // group t of its rows, one 128-byte line per 64 rank columns)
+  auto prefetch_b = [&](int tile) {
+    const int64_t row = static_cast<int64_t>(tile) * kRows + warp * 32 + 8 * t + pg;
+    if (row < a.nw)
+      for (int grp = 0; grp < a.lora_steps; ++grp)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(a.lora_b + row * a.r + grp * 64));
   };
 
   float y[2][kNT][4];
@@ -546,6 +585,7 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
   int pending = -1;
   bool dep_done = false;
 
+  prefetch_b(first.tile);
   Pos pos = first;
   uint32_t s = 0, ph = 0;
   bool alive = true;
@@ -611,6 +651,7 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
       // the share's first tile, else 1; a tile inside the share is counted and
       // finished at once, so slot 1 is free again for the next one)
       put_slot(pos.tile == first.tile ? 0 : 1, y);
+      if (it != n_mine - 1) prefetch_b(pos.tile + 1);
       if (!dep_done && pending < 0 && it != n_mine - 1) {
         pending = pos.tile;                                   // counted later
       } else {
