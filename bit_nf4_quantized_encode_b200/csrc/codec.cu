@@ -253,9 +253,11 @@ __global__ void __launch_bounds__(256) k_double_quant(const float* __restrict__ 
 
 // ------------------------------------------------------------------ dequant
 // One lane per 32 codes (16 bytes in, 64 bytes out); a 64-weight block is two
-// lanes.  Each lane takes four chunks per iteration (a grid stride apart) and
-// issues the loads of all four before expanding any.  A ragged last chunk is
-// expanded element by element.
+// lanes.  Each lane takes kDqUnroll chunks per iteration (a grid stride apart)
+// and issues the loads of all of them before expanding any: with two CTAs per
+// SM that keeps about 64 KB of codes in flight per SM, above HBM's
+// bandwidth-delay product.  A ragged last chunk is expanded element by element.
+constexpr int kDqUnroll = 8;
 __device__ __forceinline__ void dequant_chunk(const uint4 cw, uint32_t q, float c2v, float mu,
                                               const CodebookParam& cb, uint4 (&o)[4]) {
   const float c1p = block_constant(q, __fdiv_rn(c2v, 448.0f), mu);
@@ -284,13 +286,13 @@ __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ cod
   const int lane = threadIdx.x & 31;
   uint8_t* st = s_out[threadIdx.x >> 5];
   // the loop bound is uniform over the CTA, so every lane reaches the syncwarps
-  for (int64_t b0 = static_cast<int64_t>(blockIdx.x) * blockDim.x; b0 < nfull; b0 += 4 * stride) {
+  for (int64_t b0 = static_cast<int64_t>(blockIdx.x) * blockDim.x; b0 < nfull; b0 += kDqUnroll * stride) {
     const int64_t ch = b0 + threadIdx.x;
-    uint4 cw[4];
-    uint32_t qv[4];
-    float c2v[4];
+    uint4 cw[kDqUnroll];
+    uint32_t qv[kDqUnroll];
+    float c2v[kDqUnroll];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kDqUnroll; ++u) {
       const int64_t c = ch + u * stride;
       cw[u] = make_uint4(0u, 0u, 0u, 0u);
       qv[u] = 0;
@@ -302,7 +304,7 @@ __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ cod
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kDqUnroll; ++u) {
       const int64_t c = ch + u * stride;
       const int64_t wc0 = c - lane;                  // the warp's first chunk
       uint4 o[4];
