@@ -5,17 +5,17 @@
 // weight is dequantized on the fly for the matmul), bound by HBM.  Two kernels,
 // the second launched as the programmatic dependent of the first:
 //
-// k_xa_zero: partial X A^T over slices of K in fp32 (CUDA cores, CTAs that fit
-//   beside k_gemv's), and the zeroed fp32 split buffer and tile counters of
-//   k_gemv.
+// k_xa_zero: partial X A^T over slices of K in fp32 (CUDA cores), and the
+//   zeroed tile counters of k_gemv.
 //
 // k_gemv: the weight stream and the whole output.  Each CTA takes an equal,
 //   contiguous share of all (256-row tile, 256-column step) pairs, so the work
 //   is balanced whatever the shape.
-//   * A producer warp streams the [256 rows x 128 bytes] code tile
-//     (128B-swizzled) and the four [m x 64] activation boxes of each step into
-//     a 3- or 4-deep ring (TMA), and writes the step's block constants
-//     c1' = fma(e4m3(q), c2/448, mu) into the stage.
+//   * Four producer warps, one per SM sub-partition: one lane streams the
+//     [256 rows x 128 bytes] code tile (128B-swizzled) and the four [m x 64]
+//     activation boxes of each step into a 3- or 4-deep ring (TMA), and the
+//     warps write the step's block constants c1' = fma(e4m3(q), c2/448, mu)
+//     into the stage.
 //   * Eight consumer warps own 32 weight rows each.  For every 64-column block
 //     they read their rows' code bytes, turn each byte into the two bf16 levels
 //     it encodes with one shared-memory load from a 256-entry pair table (one
@@ -23,11 +23,10 @@
 //     warp MMAs (m16n8k16, bf16 in, fp32 out): a code byte is exactly one
 //     A-fragment register.  The block's product is scaled by its constant and
 //     added to fp32 registers.
-//   * A tile shared by several CTAs is summed in an fp32 split buffer; the warp
-//     whose partial completes a tile's 32 rows (a per-warp counter) adds the
-//     LoRA up-projection with warp MMAs over the staged bf16(s X A^T) and
-//     writes those rows of Y.  A tile inside one CTA's share is finished from
-//     registers.
+//   * Each warp writes its fp32 partial of a tile to one of its CTA's two
+//     slots; the warp whose partial completes a tile's 32 rows (a per-warp
+//     counter) sums the slots of the tile's CTAs, adds the LoRA up-projection
+//     with warp MMAs over the staged bf16(s X A^T) and writes those rows of Y.
 //   * The tensor core here only replaces FMAs: per weight it does 2 M FLOP.
 //     Warp MMAs are used because a skinny-N product issued as tcgen05.mma
 //     from one thread costs about 80 cycles per 128x16x16 instruction, which
@@ -682,15 +681,13 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
   (void)alive;
 }
 
-// Partial X A^T and the zeroed split buffer of k_gemv.  CTA (c, sp) computes
+// Partial X A^T and the zeroed tile counters of k_gemv.  CTA (c, sp) computes
 // LoRA columns 4c .. 4c + 3 for every token over the sp-th of nsplit slices of
 // K and writes them to part[sp] (no atomics, so nothing needs zeroing); k_gemv
-// sums the slices at its end.  Each of the 64 threads takes 8-column chunks a
-// block stride apart; the CTA reduces with warp shuffles and one exchange
-// through shared memory.  64 threads of at most 128 registers, so that a CTA
-// fits beside a k_gemv CTA on one SM: k_gemv, launched as the programmatic
-// dependent of this grid, starts streaming at once and only waits for it
-// before its first atomic.
+// sums the slices when it first finishes a tile.  Each of the 64 threads takes
+// 8-column chunks a block stride apart; the CTA reduces with warp shuffles and
+// one exchange through shared memory.  k_gemv, launched as the programmatic
+// dependent of this grid, waits for it only before it first counts a tile.
 template <int kMaxM>
 __global__ void __launch_bounds__(64, 8)
 k_xa_zero(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A, int64_t m, int64_t kw, int r,
