@@ -613,7 +613,7 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
         for (int jp = 0; jp < 2; ++jp) xv[n][jp] = lds128_if(xon[n], xs + b * kXBox + xoff[n][jp]);
       if (b == 3) {
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);                // stage fully read
+        mbar_arrive_if(lane == 0, &empty[s]);                 // stage fully read
       }
       float p[2][kNT][4];                                     // [m tile][n tile][element]
 #pragma unroll

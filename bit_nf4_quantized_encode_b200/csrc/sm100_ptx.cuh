@@ -49,6 +49,14 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
                ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Arrive from the lanes where `pred` is true, as one predicated instruction
+// (no branch, so it does not split the surrounding straight-line code).
+__device__ __forceinline__ void mbar_arrive_if(bool pred, uint64_t* bar) {
+  asm volatile("{\n\t.reg .pred p;\n\t.reg .b64 st;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+               "@p mbarrier.arrive.shared::cta.b64 st, [%0];\n\t}"
+               ::"r"(smem_u32(bar)), "r"(static_cast<uint32_t>(pred)) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
                ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
