@@ -88,8 +88,15 @@ def test_dequantize_validation_before_launch():
 def test_workspace_sizes():
     f, b = qb.qlora_linear_workspace_size(4096, 4096, 8192, 64)
     assert f >= 8192 * 64 * 6 and b >= (4096 + 4096) * 64 * 4
+    # decode shapes (M <= 16): per-warp tile counters, partial slots of at most
+    # 256 CTAs x 2 x 8 warps x 32 lanes x 16 fp32, and 16 K-slices of X A^T
     f16, b16 = qb.qlora_linear_workspace_size(22016, 8192, 16, 64)
-    assert f16 >= 16 * 22016 * 4            # split-K fp32 accumulator for decode shapes
+    tiles, steps = (22016 + 255) // 256, 8192 // 256
+    slots = min(tiles * steps, 256) * 2 * 8 * 32 * 16 * 4
+    assert f16 >= tiles * 8 * 4 + slots + 16 * 16 * 64 * 4
+    # a one-unit weight needs the slots of one CTA only
+    f_tiny, _ = qb.qlora_linear_workspace_size(256, 256, 16, 8)
+    assert 2 * 8 * 32 * 16 * 4 <= f_tiny < 2 * 2 * 8 * 32 * 16 * 4 + 16 * 16 * 64 * 4 + 1024
     with pytest.raises(qb.QloraError):
         qb.qlora_linear_workspace_size(4096, 100, 16, 64)     # cols % 64 != 0
     with pytest.raises(qb.QloraError):
