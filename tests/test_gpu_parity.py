@@ -205,6 +205,13 @@ def test_linear_decode_shapes(qb, m):
     _linear_case(qb, 392, 640, m, 64, 16.0, proj=1)
 
 
+@pytest.mark.parametrize("m,r", [(1, 72), (9, 256), (16, 136)])
+def test_linear_decode_wide_rank(qb, m, r):
+    """Decode shapes with more than one 64-column group of the rank, and a
+    partial last group: the in-kernel LoRA up-projection loops over the groups."""
+    _linear_case(qb, 392, 640, m, r, 16.0, proj=4)
+
+
 @pytest.mark.parametrize("n,k,m,r", [(392, 320, 300, 16), (256, 512, 257, 64), (136, 192, 520, 72),
                                      (512, 256, 1024, 128)])
 def test_linear_prefill_ragged(qb, n, k, m, r):
