@@ -128,7 +128,10 @@ QLORA_EXPORT qlora_status qlora_dequantize(const qlora_nf4_tensor* W, uint16_t* 
 
 /*
  * Work-buffer sizes of qlora_linear_fwd / qlora_linear_bwd for a weight of
- * shape [rows, cols], M token rows and LoRA rank r.
+ * shape [rows, cols], M token rows and LoRA rank r.  A work buffer is
+ * caller-owned device scratch: it needs no initialisation (each call clears or
+ * overwrites what it uses on its own stream), and two calls that may run at
+ * the same time must not share one.
  */
 QLORA_EXPORT qlora_status qlora_linear_workspace_size(int64_t rows, int64_t cols, int64_t M, int32_t r,
                                          size_t* fwd_bytes, size_t* bwd_bytes);
