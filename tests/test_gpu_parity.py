@@ -247,6 +247,14 @@ def test_linear_llama65b_down_projection_full_size(qb):
     _linear_case(qb, 8192, 22016, 8192, 64, 16.0, proj=6, rows_sample=rows)
 
 
+def test_linear_llama65b_q_projection_full_size(qb):
+    """8192 x 8192 (the 65B attention projections of the layer benchmark) at
+    8192 tokens, r = 64: Y and dX on 128 sampled token rows, dA and dB in full."""
+    rng = np.random.Generator(np.random.PCG64(96))
+    rows = np.sort(rng.choice(8192, 128, replace=False))
+    _linear_case(qb, 8192, 8192, 8192, 64, 16.0, proj=0, rows_sample=rows)
+
+
 def test_linear_gemv_65b_ffn(qb):
     """22016 x 8192 and 8192 x 22016 at 16 tokens, forward (decode-shaped GEMV)."""
     _linear_case(qb, 22016, 8192, 16, 64, 16.0, proj=5, check_bwd=False)
