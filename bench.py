@@ -47,26 +47,89 @@ def load_peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
-def fused_traffic():
-    """DRAM bytes (read + written) of one k_fused launch of the headline step,
-    from the committed ncu summary -- or None when that summary was not taken
-    on the fused kernel's current source (its sha256 is recorded with it)."""
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "k_fused_traffic.json")
+
+
+def _sources_digest(paths) -> str:
     import hashlib
-    summary = os.path.join(ROOT, "profiles", "k_fused_dram_traffic_llama65b_m8192.md")
-    src = os.path.join(ROOT, "bit_nf4_quantized_encode_b200", "csrc", "gemm.cu")
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def fused_traffic():
+    """DRAM bytes (read + written) of the average k_fused launch of the headline
+    step and the algorithmic bytes of the same launches, from the ncu counters
+    recorded in profiles/k_fused_traffic.json -- or (None, None) when those
+    counters were not taken on the fused kernel's current source."""
     try:
-        with open(src, "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()
-        recorded, traffic = None, None
-        with open(summary) as f:
-            for line in f:
-                if line.startswith("source_sha256"):
-                    recorded = line.split(":", 1)[1].strip()
-                elif line.startswith("traffic_bytes_per_launch:"):
-                    traffic = int(line.split(":", 1)[1].strip())
-    except (OSError, ValueError):
-        return None
-    return traffic if recorded == digest else None
+        with open(TRAFFIC_FILE) as f:
+            doc = json.load(f)
+        if doc["source_sha256"] != _sources_digest(doc["sources"]):
+            return None, None
+        n = sum(v["launches_per_step"] for v in doc["per_launch"].values())
+        traffic = sum((v["read"] + v["write"]) * v["launches_per_step"] for v in doc["per_launch"].values())
+        algo = sum(v["algorithmic"] * v["launches_per_step"] for v in doc["per_launch"].values())
+        return traffic // n, algo // n
+    except (OSError, KeyError, ValueError, ZeroDivisionError):
+        return None, None
+
+
+FUSED_SOURCES = ["bit_nf4_quantized_encode_b200/csrc/gemm.cu", "bit_nf4_quantized_encode_b200/csrc/nf4_device.cuh",
+                 "bit_nf4_quantized_encode_b200/csrc/sm100_ptx.cuh"]
+
+
+def write_traffic(csv_paths):
+    """Rebuild profiles/k_fused_traffic.json from ncu CSV logs of the --case runs
+    (one file per shape and direction, named ..._{fwd|bwd}_NxK.csv; the last
+    k_fused launch in each file is the measured one)."""
+    import csv
+    import re
+    wl = workloads.LLAMA65B
+    counts = {}
+    for p in wl.projections:
+        for d in ("fwd", "bwd"):
+            key = f"{d}_{p.n}x{p.k}"
+            counts[key] = counts.get(key, 0) + 1
+    per = {}
+    for path in csv_paths:
+        m = re.search(r"(fwd|bwd)_(\d+)x(\d+)", os.path.basename(path))
+        if not m:
+            raise SystemExit(f"cannot tell direction and shape from {path}")
+        d, n, k = m.group(1), int(m.group(2)), int(m.group(3))
+        vals = {}
+        with open(path) as f:
+            lines = [ln for ln in f if ln.startswith('"')]
+        for row in csv.DictReader(lines):
+            if "k_fused" not in row.get("Kernel Name", ""):
+                continue
+            unit = row.get("Metric Unit", "")
+            scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}.get(unit, 1)
+            vals.setdefault(row["ID"], {})[row["Metric Name"]] = float(row["Metric Value"].replace(",", "")) * scale
+        last = vals[max(vals, key=int)]
+        # activations in, packed weight, LoRA factor and its rank-r operand, bf16 output
+        algo = (2 * wl.m * (k if d == "fwd" else n) + n * k // 2 + n * k // 64 + 4 * (n * k // 16384)
+                + 2 * wl.r * (n if d == "fwd" else k) + 2 * wl.m * wl.r + 2 * wl.m * (n if d == "fwd" else k))
+        per[f"{d}_{n}x{k}"] = {"read": int(last["dram__bytes_read.sum"]), "write": int(last["dram__bytes_write.sum"]),
+                               "algorithmic": int(algo), "launches_per_step": counts[f"{d}_{n}x{k}"],
+                               "duration_ns": int(last.get("gpu__time_duration.sum", 0))}
+    doc = {"what": "DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one k_fused launch per shape "
+                   "and direction, LLaMA-65B layer projections at 8192 tokens, LoRA r 64; bench.py reads it for "
+                   "roofline.traffic while source_sha256 matches the listed sources",
+           "kernel": "k_fused", "workload": wl.name, "sources": FUSED_SOURCES,
+           "source_sha256": _sources_digest(FUSED_SOURCES),
+           "command": "python bench.py --case fused_{fwd,bwd} --case-n N --case-k K --case-m 8192 --case-iters 1; "
+                      "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
+                      "--clock-control none -k regex:k_fused --csv --log-file traffic_{fwd,bwd}_NxK.csv <same command>",
+           "per_launch": per}
+    missing = set(counts) - set(per)
+    if missing:
+        raise SystemExit(f"no capture for {sorted(missing)}")
+    with open(TRAFFIC_FILE, "w") as f:
+        json.dump(doc, f, indent=1)
+    print(f"wrote {TRAFFIC_FILE}")
 
 
 # ---------------------------------------------------------------------------- clocks
@@ -334,8 +397,10 @@ def secondary(qb, torch, device, peaks):
 
 
 def cpu_oracle_sample(wl, m_sample: int, projs_idx=None) -> dict:
-    """The oracle (as it stands) on a bounded sample of the same workload: all
-    weights dequantized by the C oracle, then fwd + bwd of m_sample tokens."""
+    """The oracle (as it stands) on a bounded sample of a layer workload: the
+    weights dequantized by the C oracle, then fwd + bwd of m_sample tokens in
+    float64.  Returns the measured seconds of both parts (quantization, a model
+    load, is timed apart) and the TFLOP/s of the sample."""
     import oracle
     t_quant = time.time()
     qts = []
@@ -346,28 +411,203 @@ def cpu_oracle_sample(wl, m_sample: int, projs_idx=None) -> dict:
         qts.append((i, p, oracle.quantize(workloads.bf16_bits(w))))
         del w
     t_quant = time.time() - t_quant
-    t0 = time.time()
-    flops = 0
+    t_deq, t_mm, flops = 0.0, 0.0, 0
     for i, p, qt in qts:
-        Wd = oracle.dequant_tensor(qt)
         X = workloads.activations(wl.m, p.k, i)[:m_sample].float().numpy()
         dY = workloads.grad_output(wl.m, p.n, i)[:m_sample].float().numpy()
         A = workloads.lora_a(wl.r, p.k, i).float().numpy()
         B = workloads.lora_b(p.n, wl.r, i).float().numpy()
+        t0 = time.time()
+        Wd = oracle.dequant_tensor(qt)
+        t1 = time.time()
         oracle.linear_fwd(Wd, X, A, B, wl.s)
         oracle.linear_bwd(Wd, X, dY, A, B, wl.s)
+        t2 = time.time()
+        t_deq += t1 - t0
+        t_mm += t2 - t1
         flops += workloads.linear_flops(p.n, p.k, m_sample, wl.r)["total"]
-    t = time.time() - t0
-    try:
-        from threadpoolctl import threadpool_info
-        blas = max([x.get("num_threads", 1) for x in threadpool_info()] + [1])
-    except Exception:
-        blas = os.cpu_count()
-    cores = max(blas, int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1)))
-    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "seconds": round(t, 2), "setup_quantize_seconds": round(t_quant, 2),
+    t = t_deq + t_mm
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            "seconds": round(t, 2), "dequant_seconds": round(t_deq, 2), "matmul_seconds": round(t_mm, 3),
+            "setup_quantize_seconds": round(t_quant, 2),
             "sample": f"{m_sample} of {wl.m} tokens of each of {len(qts)} projections of {wl.name}: "
                       f"C-oracle dequant of the full weights + float64 numpy fwd+bwd"}
+
+
+def cpu_baseline(slice5: int = 512) -> dict:
+    """The oracle as it stands, timed on this host's cores (OpenMP in the C codec,
+    the BLAS threads in numpy), on the five workloads:
+      1 (tiny layer), 2 (4096^2 codec) and 4 (65B FFN decode forward) in full;
+      3 (LLaMA-7B 7 projections, 8192 tokens) in full;
+      5 (LLaMA-65B layer) on a slice of `slice5` tokens of every projection,
+        extrapolated to 8192 tokens as dequant + (8192 / slice) x the slice's
+        matmuls -- labelled as such.
+    The headline value is workload 5's extrapolated TFLOP/s."""
+    import oracle
+    out = {}
+    # 1: quantize + forward + backward of the tiny layer
+    wl = workloads.TINY
+    p = wl.projections[0]
+    w = workloads.bf16_bits(workloads.weight((p.n, p.k)))
+    X, A = workloads.activations(wl.m, p.k).float().numpy(), workloads.lora_a(wl.r, p.k).float().numpy()
+    B, dY = workloads.lora_b(p.n, wl.r).float().numpy(), workloads.grad_output(wl.m, p.n).float().numpy()
+    t0 = time.time()
+    for _ in range(10):
+        Wd = oracle.dequant_tensor(oracle.quantize(w))
+        oracle.linear_fwd(Wd, X, A, B, wl.s)
+        oracle.linear_bwd(Wd, X, dY, A, B, wl.s)
+    out["1_" + wl.name] = {"us_per_call": round((time.time() - t0) / 10 * 1e6, 1),
+                           "what": "quantize + dequant + fwd + bwd, in full"}
+    # 2: encode + double quant, then dequant, of the 4096^2 weight with outliers
+    wbits = workloads.bf16_bits(workloads.weight((4096, 4096), proj=0, outliers=True))
+    t0 = time.time()
+    qt = oracle.quantize(wbits)
+    t1 = time.time()
+    oracle.dequant_tensor(qt)
+    t2 = time.time()
+    sz = oracle.storage_bytes(4096 * 4096)
+    nbytes = 4096 * 4096 * 2 + sz["codes"] + sz["absmax_q"] + sz["absmax_c2"] + sz["mean"]
+    out["2_" + workloads.CODEC_4096.name] = {"encode_GB/s": round(nbytes / (t1 - t0) / 1e9, 3),
+                                             "dequant_GB/s": round(nbytes / (t2 - t1) / 1e9, 3),
+                                             "what": "in full"}
+    del wbits, qt
+    # 4: decode-shaped forward on the 65B FFN weights (dequant + fwd per call)
+    g = {}
+    for j, pj in enumerate(workloads.GEMV65B.projections):
+        qt = oracle.quantize(workloads.bf16_bits(workloads.weight((pj.n, pj.k), proj=20 + j)))
+        szg = oracle.storage_bytes(pj.n * pj.k)
+        A = workloads.lora_a(64, pj.k, 30).float().numpy()
+        B = workloads.lora_b(pj.n, 64, 30).float().numpy()
+        for m in workloads.GEMV65B.token_counts:
+            X = workloads.activations(m, pj.k, 31).float().numpy()
+            t0 = time.time()
+            Wd = oracle.dequant_tensor(qt)
+            oracle.linear_fwd(Wd, X, A, B, 0.25)
+            t = time.time() - t0
+            nb = (szg["codes"] + szg["absmax_q"] + szg["absmax_c2"] + szg["mean"] + (A.size + B.size) * 2
+                  + m * pj.k * 2 + m * pj.n * 2)
+            g[f"{pj.n}x{pj.k}_m{m}"] = round(nb / t / 1e9, 3)
+        del qt
+    out["4_" + workloads.GEMV65B.name] = {"GB/s": g, "what": "dequant + fwd per call, in full"}
+    # 3: LLaMA-7B projections, all 8192 tokens
+    r3 = cpu_oracle_sample(workloads.LLAMA7B, workloads.LLAMA7B.m)
+    out["3_" + workloads.LLAMA7B.name] = {"TFLOP/s": round(r3["value"], 5), "seconds": r3["seconds"],
+                                          "what": "dequant + fwd + bwd, all 8192 tokens (in full)"}
+    # 5: the headline layer on a token slice, extrapolated
+    wl5 = workloads.LLAMA65B
+    r5 = cpu_oracle_sample(wl5, slice5)
+    t_full = r5["dequant_seconds"] + r5["matmul_seconds"] * wl5.m / slice5
+    flops5 = sum(workloads.linear_flops(p.n, p.k, wl5.m, wl5.r)["total"] for p in wl5.projections)
+    value = flops5 / t_full / 1e12
+    out["5_" + wl5.name] = {"TFLOP/s_extrapolated": round(value, 5), "slice_TFLOP/s": round(r5["value"], 5),
+                            "seconds": r5["seconds"],
+                            "what": f"{slice5}-token slice of every projection, extrapolated to {wl5.m} tokens"}
+    return {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{wl5.name}: {slice5} of {wl5.m} tokens of all 7 projections (C-oracle dequant of the "
+                      f"full weights + float64 numpy fwd+bwd), extrapolated to {wl5.m} tokens; the other "
+                      f"workloads under 'workloads'",
+            "workloads": out}
+
+
+def time_layer(qb, torch, wl, projs, steps: int, pg=None, device=None, with_clocks=False):
+    """Times `steps` steps of a layer workload (inputs resident in HBM) with CUDA
+    events on the launching stream, every fused dequant-GEMM launch bracketed by
+    its own pair of events.  Returns the step time (max over ranks), the fused
+    launches' durations, the kernel-launch count and the clocks seen."""
+    gemm_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(2 * len(projs) * steps)]
+    for a, b in gemm_events:          # torch creates the CUDA event on first record
+        a.record()
+        b.record()
+    ev_stack = list(reversed(gemm_events))
+    clocks = ClockSampler(device.index) if with_clocks else None
+    barrier(pg, device)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+    launches0 = qb.qlora_kernel_launches()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        run_step(qb, wl, projs, events=ev_stack)
+    e1.record()
+    torch.cuda.synchronize()
+    launches = qb.qlora_kernel_launches() - launches0
+    barrier(pg, device)
+    clk = clocks.stop() if clocks else None
+    t_local = e0.elapsed_time(e1) / 1e3
+    t = max_over_ranks(pg, t_local, device)
+    gemm_ms = [a.elapsed_time(b) for a, b in gemm_events]
+    return dict(t=t, t_local=t_local, gemm_ms=gemm_ms, launches=launches, clocks=clk)
+
+
+def layer_summary(wl, timing, steps, peaks, world=1) -> dict:
+    flops_step, flops_fused_step = layer_flops(wl)
+    value = world * steps * flops_step / timing["t"] / 1e12
+    fused_avg_s = sum(timing["gemm_ms"]) / len(timing["gemm_ms"]) / 1e3
+    achieved = flops_fused_step / (2 * len(wl.projections)) / fused_avg_s / 1e12
+    sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    return {"TFLOP/s": round(value, 2), "ms_per_step": round(timing["t"] / steps * 1e3, 3),
+            "frac_sustained": round(value / sus, 4), "frac_burst": round(value / peaks["bf16_tflops"], 4),
+            "k_fused_TFLOP/s": round(achieved, 1), "k_fused_frac_sustained": round(achieved / sus, 4),
+            "k_fused_frac_burst": round(achieved / peaks["bf16_tflops"], 4),
+            "k_fused_share": round(sum(timing["gemm_ms"]) / 1e3 / timing["t_local"], 4),
+            "flops_per_step": flops_step, "steps": steps}
+
+
+def tiny_layer_us(qb, torch, device) -> dict:
+    """The tiny layer (256 x 256, 16 tokens, r 8): launch-bound, so reported in
+    microseconds per call, graph-timed over 20 back-to-back calls each."""
+    wl = workloads.TINY
+    p = wl.projections[0]
+    w = workloads.weight((p.n, p.k)).to(device)
+    qt = qb.qlora_quantize_nf4_dq(w)
+    X, dY = workloads.activations(wl.m, p.k).to(device), workloads.grad_output(wl.m, p.n).to(device)
+    A, B = workloads.lora_a(wl.r, p.k).to(device), workloads.lora_b(p.n, wl.r).to(device)
+    fw, bw = qb.qlora_linear_workspace_size(p.n, p.k, wl.m, wl.r)
+    wsf = torch.empty(fw, dtype=torch.uint8, device=device)
+    wsb = torch.empty(bw, dtype=torch.uint8, device=device)
+    wsq = torch.empty(qb.qlora_nf4_sizes(p.n, p.k)["workspace"], dtype=torch.uint8, device=device)
+    Y = torch.empty(wl.m, p.n, dtype=torch.bfloat16, device=device)
+    XA = torch.empty(wl.m, wl.r, dtype=torch.float32, device=device)
+    dX = torch.empty(wl.m, p.k, dtype=torch.bfloat16, device=device)
+    dA = torch.empty(wl.r, p.k, dtype=torch.float32, device=device)
+    dB = torch.empty(p.n, wl.r, dtype=torch.float32, device=device)
+    ops = {
+        "quantize": lambda: qb.qlora_quantize_nf4_dq(w, out=qt, workspace=wsq),
+        "fwd": lambda: qb.qlora_linear_fwd(qt, X, A, B, wl.s, Y=Y, XA=XA, workspace=wsf),
+        "bwd": lambda: qb.qlora_linear_bwd(qt, X, dY, A, B, wl.s, XA=XA, dX=dX, dA=dA, dB=dB, workspace=wsb),
+    }
+    out = {}
+    for name, fn in ops.items():
+        out[f"{name}_us"] = round(graph_time(torch, fn, 20, 5) * 1e6, 2)
+    return out
+
+
+def graph_time(torch, fn, calls: int, replays: int) -> float:
+    """Seconds per call of `fn`, captured `calls` times in one CUDA graph and
+    replayed `replays` times (no host launch gaps)."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(calls):
+                fn()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(replays):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) / 1e3 / (calls * replays)
 
 
 def bench_ours(args):
@@ -388,29 +628,8 @@ def bench_ours(args):
 
     # timed region: K steps, fused-GEMM launches bracketed by events for the roofline
     K = args.steps
-    gemm_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(2 * len(projs) * K)]
-    for a, b in gemm_events:          # torch creates the CUDA event on first record
-        a.record()
-        b.record()
-    ev_stack = list(reversed(gemm_events))
-    clocks = ClockSampler(device.index)
-    barrier(pg, device)
-    torch.cuda.synchronize()
-    clocks.start()
-    launches0 = qb.qlora_kernel_launches()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(K):
-        run_step(qb, wl, projs, events=ev_stack)
-    e1.record()
-    torch.cuda.synchronize()
-    launches = qb.qlora_kernel_launches() - launches0
-    barrier(pg, device)
-    clk = clocks.stop()
-    t_local = e0.elapsed_time(e1) / 1e3
-    t = max_over_ranks(pg, t_local, device)
-    gemm_ms = [a.elapsed_time(b) for a, b in gemm_events]
+    tm = time_layer(qb, torch, wl, projs, K, pg, device, with_clocks=True)
+    t, t_local, gemm_ms, launches, clk = tm["t"], tm["t_local"], tm["gemm_ms"], tm["launches"], tm["clocks"]
 
     # end to end: host inputs -> device -> fwd+bwd -> gradients back to host
     Ke = max(2, min(K, 5))
@@ -432,6 +651,21 @@ def bench_ours(args):
     h2d = sum(st["X"].numel() * 2 + st["dY"].numel() * 2 for st in projs)
     d2h = sum(st["dA"].numel() * 4 + st["dB"].numel() * 4 for st in projs)
     assert qb.qlora_read_device_errors() == 0
+    del projs
+
+    # the other layer workload (LLaMA-7B, 7 projections, 8192 tokens) and the tiny layer
+    others = {}
+    if not args.skip_secondary:
+        wl3 = workloads.LLAMA7B
+        projs3 = prepare_layer(qb, torch, wl3, device)
+        for _ in range(3):
+            run_step(qb, wl3, projs3)
+        K3 = max(5, K // 2)
+        tm3 = time_layer(qb, torch, wl3, projs3, K3, pg, device)
+        others["3_" + wl3.name] = layer_summary(wl3, tm3, K3, peaks, world)
+        del projs3
+        others["1_" + workloads.TINY.name] = tiny_layer_us(qb, torch, device)
+        assert qb.qlora_read_device_errors() == 0
     if pg is not None:                 # every rank takes the same collective steps
         barrier(pg, device)
         pg.destroy_process_group()
@@ -441,8 +675,9 @@ def bench_ours(args):
     value = world * K * flops_step / t / 1e12
     peak_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     fused_avg_s = sum(gemm_ms) / len(gemm_ms) / 1e3
-    fused_flops_launch = flops_fused_step / (2 * len(projs))
+    fused_flops_launch = flops_fused_step / (2 * len(wl.projections))
     achieved = fused_flops_launch / fused_avg_s / 1e12
+    traffic, algo_bytes = fused_traffic()
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(t / K * 1e3, 3), "higher_is_better": True,
@@ -459,15 +694,23 @@ def bench_ours(args):
         "roofline": {"bound": "tensor", "kernel": "k_fused (dequant-GEMM fwd and bwd-dX)",
                      "achieved": round(achieved, 1), "peak": peak_t, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_t, 4), "peak_kind": f"{peak_kind} sustained bf16",
-                     "traffic": fused_traffic(), "traffic_unit": "bytes per launch (ncu, profiles/)",
+                     "frac_of_burst_peak": round(achieved / peaks["bf16_tflops"], 4),
+                     "burst_peak": peaks["bf16_tflops"],
+                     "traffic": traffic,
+                     "traffic_unit": "DRAM bytes per average launch (ncu counters, profiles/k_fused_traffic.json; "
+                                     "null when taken on other source)",
+                     "algorithmic_bytes": algo_bytes,
+                     "traffic_over_algorithmic": round(traffic / algo_bytes, 3) if traffic and algo_bytes else None,
                      "avg_launch_ms": round(fused_avg_s * 1e3, 4),
                      "share_of_step": round(sum(gemm_ms) / 1e3 / t_local, 4)},
         "clocks": clk,
     }
+    if others:
+        line["workloads"] = others
     if not args.skip_secondary:
         line["secondary"] = secondary(qb, torch, device, peaks)
     if not args.skip_cpu:
-        line["cpu_baseline"] = cpu_oracle_sample(wl, m_sample=args.cpu_tokens)
+        line["cpu_baseline"] = cpu_baseline(slice5=args.cpu_tokens)
     print(json.dumps(line), flush=True)
 
 
@@ -543,7 +786,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--skip-secondary", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
-    ap.add_argument("--cpu-tokens", type=int, default=64, help="token sample of the CPU-oracle baseline")
+    ap.add_argument("--cpu-tokens", type=int, default=512,
+                    help="token slice of the LLaMA-65B layer in the CPU-oracle baseline")
     ap.add_argument("--ref-tokens", type=int, default=16, help="token sample per reference-arm step")
     ap.add_argument("--case", choices=["fused_fwd", "fused_bwd", "encode", "dequant"],
                     help="run one operation on a small case (for profiler captures) and exit")
@@ -551,7 +795,12 @@ def main():
     ap.add_argument("--case-k", type=int, default=8192)
     ap.add_argument("--case-m", type=int, default=4096)
     ap.add_argument("--case-iters", type=int, default=3)
+    ap.add_argument("--write-traffic", nargs="+", metavar="CSV",
+                    help="rebuild profiles/k_fused_traffic.json from ncu CSV logs of the --case runs and exit")
     args = ap.parse_args()
+    if args.write_traffic:
+        write_traffic(args.write_traffic)
+        return
     if args.case:
         run_case(args)
         return

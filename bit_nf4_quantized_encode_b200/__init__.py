@@ -70,11 +70,13 @@ _lib.qlora_kernel_launches.argtypes = []
 _lib.qlora_kernel_launches.restype = ctypes.c_uint64
 _lib.qlora_time_next_gemm.argtypes = [_vp, _vp]
 _lib.qlora_time_next_gemm.restype = ctypes.c_int
+_lib.qlora_selftest_bounded_wait.argtypes = [_i64, _vp, _vp]
+_lib.qlora_selftest_bounded_wait.restype = ctypes.c_int
 
 EXPORTED = ["qlora_status_string", "qlora_get_codebook", "qlora_nf4_sizes", "qlora_quantize_nf4_dq",
             "qlora_dequantize", "qlora_linear_workspace_size", "qlora_linear_fwd",
             "qlora_linear_bwd", "qlora_read_device_errors", "qlora_kernel_launches",
-            "qlora_time_next_gemm", "qlora_quantize_nf4_dq_noalloc"]
+            "qlora_time_next_gemm", "qlora_quantize_nf4_dq_noalloc", "qlora_selftest_bounded_wait"]
 
 # Largest weight the allocation-free quantize variant accepts.
 NOALLOC_MAX_ELEMENTS = 134217728
@@ -157,6 +159,17 @@ def empty_nf4(rows: int, cols: int, device) -> NF4Tensor:
                      rows=rows, cols=cols)
 
 
+def _check_out_matches(W: torch.Tensor, out: NF4Tensor):
+    """The C entry points take the shape from `out` alone and read that many
+    weights from W: refuse a destination that describes another tensor."""
+    if out.rows * out.cols != W.numel():
+        raise ValueError(f"out describes {out.rows}x{out.cols} weights, W has {W.numel()}")
+    for name, t in (("codes", out.codes), ("absmax_q", out.absmax_q), ("absmax_c2", out.absmax_c2),
+                    ("absmax_mean", out.absmax_mean)):
+        if t.device != W.device:
+            raise ValueError(f"out.{name} is on {t.device}, W on {W.device}")
+
+
 def qlora_quantize_nf4_dq(W: torch.Tensor, out: NF4Tensor | None = None,
                           workspace: torch.Tensor | None = None) -> NF4Tensor:
     """Blockwise NF4 encode + double quantization of a bf16 [rows, cols] weight."""
@@ -164,6 +177,7 @@ def qlora_quantize_nf4_dq(W: torch.Tensor, out: NF4Tensor | None = None,
     rows, cols = (W.shape[0], W.shape[1]) if W.dim() == 2 else (1, W.numel())
     if out is None:
         out = empty_nf4(rows, cols, W.device)
+    _check_out_matches(W, out)
     need = qlora_nf4_sizes(rows, cols)["workspace"]
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
@@ -177,6 +191,7 @@ def qlora_quantize_nf4_dq_noalloc(W: torch.Tensor, out: NF4Tensor) -> NF4Tensor:
     """Same result as qlora_quantize_nf4_dq, with the library's built-in scratch
     instead of a work buffer (for callers that cannot allocate; see qlora.h)."""
     _need_bf16_cuda("W", W)
+    _check_out_matches(W, out)
     c = out.c_struct()
     _check(_lib.qlora_quantize_nf4_dq_noalloc(_ptr(W), ctypes.byref(c), _stream(W.device)),
            "qlora_quantize_nf4_dq_noalloc")
@@ -252,6 +267,14 @@ def qlora_read_device_errors(clear: bool = True) -> int:
     _check(_lib.qlora_read_device_errors(ctypes.byref(v), 1 if clear else 0),
            "qlora_read_device_errors")
     return v.value
+
+
+def qlora_selftest_bounded_wait(limit_cycles: int, outcome: torch.Tensor | None = None) -> None:
+    """Launch the failure-path self-test: one CTA whose bounded mbarrier wait
+    must give up after `limit_cycles` SM cycles (see qlora.h)."""
+    _check(_lib.qlora_selftest_bounded_wait(int(limit_cycles), _ptr(outcome),
+                                            _stream(outcome.device if outcome is not None else None)),
+           "qlora_selftest_bounded_wait")
 
 
 def qlora_kernel_launches() -> int:

@@ -15,6 +15,7 @@
 #include "codec.h"
 #include "gemm.h"
 #include "gemv.h"
+#include "internal.h"
 #include "nf4_tables.h"
 #include "qlora.h"
 
@@ -40,12 +41,6 @@ struct DeviceInfo {
 std::mutex g_mu;
 std::atomic<uint64_t> g_launches{0};
 thread_local cudaEvent_t t_gemm_start = nullptr, t_gemm_stop = nullptr;
-
-// Counts one kernel launch when it succeeded.
-cudaError_t counted(cudaError_t e, int n = 1) {
-  if (e == cudaSuccess) g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed);
-  return e;
-}
 
 cudaError_t fused_timed(FusedDir dir, int bn, const FusedArgs& fa, const CUtensorMap& act,
                         const CUtensorMap& lora, int num_sms, cudaStream_t cs) {
@@ -148,18 +143,6 @@ int balanced_splits(int tiles, int ksteps, int sms) {
   return best;
 }
 
-qlora_status check_tensor(const qlora_nf4_tensor* t) {
-  if (!t) return QLORA_ERR_NULL;
-  if (t->rows < 0 || t->cols < 0 || t->rows > kMaxDim || t->cols > kMaxDim) return QLORA_ERR_SHAPE;
-  if (t->blocksize != kBlock || t->blocksize2 != kBlock2) return QLORA_ERR_UNSUPPORTED;
-  if (t->rows * t->cols == 0) return QLORA_OK;
-  if (!t->codes || !t->absmax_q || !t->absmax_c2 || !t->absmax_mean) return QLORA_ERR_NULL;
-  if (!aligned16(t->codes) || !aligned16(t->absmax_q) || !aligned16(t->absmax_c2) ||
-      !aligned16(t->absmax_mean))
-    return QLORA_ERR_ALIGN;
-  return QLORA_OK;
-}
-
 CodebookParam codebook_param() {
   CodebookParam cb;
   const Nf4Tables& t = nf4_tables();
@@ -260,6 +243,31 @@ qlora_status run_skinny(bool a_mn, bool b_mn, const CUtensorMap& am, const CUten
 }
 
 }  // namespace
+
+cudaError_t counted(cudaError_t e, int n) {
+  if (e == cudaSuccess) g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed);
+  return e;
+}
+
+qlora_status check_tensor(const qlora_nf4_tensor* t) {
+  if (!t) return QLORA_ERR_NULL;
+  if (t->rows < 0 || t->cols < 0 || t->rows > kMaxDim || t->cols > kMaxDim) return QLORA_ERR_SHAPE;
+  if (t->blocksize != kBlock || t->blocksize2 != kBlock2) return QLORA_ERR_UNSUPPORTED;
+  if (t->rows * t->cols == 0) return QLORA_OK;
+  if (!t->codes || !t->absmax_q || !t->absmax_c2 || !t->absmax_mean) return QLORA_ERR_NULL;
+  if (!aligned16(t->codes) || !aligned16(t->absmax_q) || !aligned16(t->absmax_c2) ||
+      !aligned16(t->absmax_mean))
+    return QLORA_ERR_ALIGN;
+  return QLORA_OK;
+}
+
+qlora_status device_error_flag(uint32_t** flag) {
+  DeviceInfo d;
+  const qlora_status st = device_info(&d);
+  if (st == QLORA_OK) *flag = d.err;
+  return st;
+}
+
 }  // namespace qlora
 
 using namespace qlora;
@@ -448,11 +456,11 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor* W, const uint16_t* X, int6
     return st;
   // 2) bf16(s XA), zero-padded to a multiple of 64 columns, as the LoRA k-step operand;
   //    XA itself (fp32, unscaled) for the backward pass
-  if (counted(launch_convert_bf16(xa_acc, sh.m, sh.rpad, sh.rpad, sh.rpad, s, sxa, sh.rpad, cs)) !=
+  if (counted(launch_convert_bf16(xa_acc, sh.m, sh.rpad, sh.rpad, sh.rpad, s, sxa, sh.rpad, d.num_sms, cs)) !=
       cudaSuccess)
     return QLORA_ERR_CUDA;
   if (XA_out &&
-      counted(launch_convert_f32(xa_acc, sh.m, sh.r, sh.rpad, 1.0f, false, XA_out, sh.r, cs)) !=
+      counted(launch_convert_f32(xa_acc, sh.m, sh.r, sh.rpad, 1.0f, false, XA_out, sh.r, d.num_sms, cs)) !=
           cudaSuccess)
     return QLORA_ERR_CUDA;
 
@@ -515,7 +523,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor* W, const uint16_t* X, cons
     return QLORA_ERR_CUDA;
   if ((st = run_skinny(false, true, dy_k, b_mn, sh.m, sh.r, sh.rows, g_acc, sh.rpad, d, cs)) != QLORA_OK)
     return st;
-  if (counted(launch_convert_bf16(g_acc, sh.m, sh.rpad, sh.rpad, sh.rpad, s, sg, sh.rpad, cs)) !=
+  if (counted(launch_convert_bf16(g_acc, sh.m, sh.rpad, sh.rpad, sh.rpad, s, sg, sh.rpad, d.num_sms, cs)) !=
       cudaSuccess)
     return QLORA_ERR_CUDA;
 
@@ -557,7 +565,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor* W, const uint16_t* X, cons
     if (fused_timed(FusedDir::kBwd, bn, fa, dy_act, sg_map, d.num_sms, cs) != cudaSuccess)
       return QLORA_ERR_CUDA;
     if (fa.splits > 1 &&
-        counted(launch_convert_bf16(dx_acc, sh.m, sh.cols, sh.cols, sh.cols, 1.0f, dX, sh.cols, cs)) !=
+        counted(launch_convert_bf16(dx_acc, sh.m, sh.cols, sh.cols, sh.cols, 1.0f, dX, sh.cols, d.num_sms, cs)) !=
             cudaSuccess)
       return QLORA_ERR_CUDA;
   }
@@ -565,13 +573,13 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor* W, const uint16_t* X, cons
   // 4) LoRA gradients.  Few tokens: fp32 on CUDA cores from the fp32 G and XA.
   if (sh.decode) {
     if (counted(launch_small_grads(g_acc, sh.rpad, xa, ld_xa, X, dY, sh.m, sh.rows, sh.cols, sh.r, s,
-                                   dA, dB, cs)) != cudaSuccess)
+                                   dA, dB, d.num_sms, cs)) != cudaSuccess)
       return QLORA_ERR_CUDA;
     return QLORA_OK;
   }
   //    Many tokens: tcgen05 contractions over the tokens with bf16 operands.
   //    dB = dY^T (s XA)  ([rows, r]; both operands MN-major)
-  if (counted(launch_convert_bf16(xa, sh.m, sh.r, ld_xa, sh.rpad, s, sxa, sh.rpad, cs)) != cudaSuccess)
+  if (counted(launch_convert_bf16(xa, sh.m, sh.r, ld_xa, sh.rpad, s, sxa, sh.rpad, d.num_sms, cs)) != cudaSuccess)
     return QLORA_ERR_CUDA;
   CUtensorMap dy_mn, sxa_mn;
   if (!make_map(&dy_mn, dY, sh.rows, sh.m, sh.rows * 2, 64) ||
@@ -586,9 +594,9 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor* W, const uint16_t* X, cons
     return QLORA_ERR_CUDA;
   if ((st = run_skinny(true, true, x_mn, sg_mn, sh.cols, sh.r, sh.m, da_acc, sh.rpad, d, cs)) != QLORA_OK)
     return st;
-  if (counted(launch_convert_f32(db_acc, sh.rows, sh.r, sh.rpad, 1.0f, false, dB, sh.r, cs)) != cudaSuccess)
+  if (counted(launch_convert_f32(db_acc, sh.rows, sh.r, sh.rpad, 1.0f, false, dB, sh.r, d.num_sms, cs)) != cudaSuccess)
     return QLORA_ERR_CUDA;
-  if (counted(launch_convert_f32(da_acc, sh.cols, sh.r, sh.rpad, 1.0f, true, dA, sh.cols, cs)) != cudaSuccess)
+  if (counted(launch_convert_f32(da_acc, sh.cols, sh.r, sh.rpad, 1.0f, true, dA, sh.cols, d.num_sms, cs)) != cudaSuccess)
     return QLORA_ERR_CUDA;
   return QLORA_OK;
 }

@@ -643,32 +643,32 @@ cudaError_t launch_skinny(bool a_mn, bool b_mn, const SkinnyArgs& args, const CU
 }
 
 cudaError_t launch_convert_bf16(const float* in, int64_t rows, int64_t cols_in, int64_t ld_in,
-                                int64_t cols_out, float scale, uint16_t* out, int64_t ld_out,
+                                int64_t cols_out, float scale, uint16_t* out, int64_t ld_out, int num_sms,
                                 cudaStream_t stream) {
   const int64_t n = rows * cols_out;
   if (n == 0) return cudaSuccess;
-  k_convert<uint16_t><<<grid_for(n, 148), 256, 0, stream>>>(in, rows, cols_in, ld_in, cols_out, scale,
+  k_convert<uint16_t><<<grid_for(n, num_sms), 256, 0, stream>>>(in, rows, cols_in, ld_in, cols_out, scale,
                                                              out, ld_out);
   return cudaGetLastError();
 }
 
 cudaError_t launch_convert_f32(const float* in, int64_t rows, int64_t cols, int64_t ld_in, float scale,
-                               bool transpose, float* out, int64_t ld_out, cudaStream_t stream) {
+                               bool transpose, float* out, int64_t ld_out, int num_sms, cudaStream_t stream) {
   const int64_t n = rows * cols;
   if (n == 0) return cudaSuccess;
   if (transpose)
-    k_convert_t<<<grid_for(n, 148), 256, 0, stream>>>(in, rows, cols, ld_in, scale, out, ld_out);
+    k_convert_t<<<grid_for(n, num_sms), 256, 0, stream>>>(in, rows, cols, ld_in, scale, out, ld_out);
   else
-    k_convert<float><<<grid_for(n, 148), 256, 0, stream>>>(in, rows, cols, ld_in, cols, scale, out, ld_out);
+    k_convert<float><<<grid_for(n, num_sms), 256, 0, stream>>>(in, rows, cols, ld_in, cols, scale, out, ld_out);
   return cudaGetLastError();
 }
 
 cudaError_t launch_small_grads(const float* G, int64_t ld_g, const float* XA, int64_t ld_xa,
                                const uint16_t* X, const uint16_t* dY, int64_t M, int64_t rows,
-                               int64_t cols, int r, float s, float* dA, float* dB,
+                               int64_t cols, int r, float s, float* dA, float* dB, int num_sms,
                                cudaStream_t stream) {
   const int64_t n = static_cast<int64_t>(r) * (cols + rows);
-  k_small_grads<<<grid_for(n, 148), 256, 0, stream>>>(G, ld_g, XA, ld_xa, X, dY, M, rows, cols, r, s,
+  k_small_grads<<<grid_for(n, num_sms), 256, 0, stream>>>(G, ld_g, XA, ld_xa, X, dY, M, rows, cols, r, s,
                                                       dA, dB);
   return cudaGetLastError();
 }

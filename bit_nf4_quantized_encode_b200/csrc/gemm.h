@@ -64,17 +64,18 @@ cudaError_t launch_skinny(bool a_mn_major, bool b_mn_major, const SkinnyArgs& ar
 // out[i * ld_out + j] = T(scale * in[i * ld_in + j]) for j < cols_in, 0 for
 // cols_in <= j < cols_out (i < rows); T is bf16 or fp32.  With `transpose`
 // the element goes to out[j * ld_out + i] instead (cols_out == cols_in).
+// Grids are at most 8 CTAs of 256 threads per SM (num_sms: the device's SM count).
 cudaError_t launch_convert_bf16(const float* in, int64_t rows, int64_t cols_in, int64_t ld_in,
-                                int64_t cols_out, float scale, uint16_t* out, int64_t ld_out,
+                                int64_t cols_out, float scale, uint16_t* out, int64_t ld_out, int num_sms,
                                 cudaStream_t stream);
 cudaError_t launch_convert_f32(const float* in, int64_t rows, int64_t cols, int64_t ld_in, float scale,
-                               bool transpose, float* out, int64_t ld_out, cudaStream_t stream);
+                               bool transpose, float* out, int64_t ld_out, int num_sms, cudaStream_t stream);
 
 // LoRA gradients for few tokens (M <= 16), fp32 throughout on CUDA cores:
 //   dA[j, k] = s * sum_m G[m, j] X[m, k];   dB[n, j] = s * sum_m dY[m, n] XA[m, j]
 cudaError_t launch_small_grads(const float* G, int64_t ld_g, const float* XA, int64_t ld_xa,
                                const uint16_t* X, const uint16_t* dY, int64_t M, int64_t rows,
-                               int64_t cols, int r, float s, float* dA, float* dB,
+                               int64_t cols, int r, float s, float* dA, float* dB, int num_sms,
                                cudaStream_t stream);
 
 }  // namespace qlora

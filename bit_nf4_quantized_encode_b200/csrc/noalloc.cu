@@ -23,6 +23,7 @@
 #include <mutex>
 
 #include "codec.h"
+#include "internal.h"
 #include "nf4_tables.h"
 #include "qlora.h"
 
@@ -72,23 +73,21 @@ using namespace qlora;
 
 extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const uint16_t* W, const qlora_nf4_tensor* out,
                                                        qlora_stream_t stream) {
-  if (!out) return QLORA_ERR_NULL;
-  if (out->rows < 0 || out->cols < 0) return QLORA_ERR_SHAPE;
-  if (out->blocksize != 64 || out->blocksize2 != 256) return QLORA_ERR_UNSUPPORTED;
-  if (out->rows > 0 && out->cols > QLORA_NOALLOC_MAX_ELEMENTS / out->rows) return QLORA_ERR_WORKSPACE;
+  // the descriptor checks of qlora_quantize_nf4_dq, in the same order, so the
+  // same bad call gets the same status from both entry points
+  qlora_status st = check_tensor(out);
+  if (st != QLORA_OK) return st;
   const int64_t numel = out->rows * out->cols;
   if (numel == 0) return QLORA_OK;
+  if (!W) return QLORA_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(W) & 15u) != 0) return QLORA_ERR_ALIGN;
+  // in place of the work-buffer size check: the built-in scratch's limit
   if (numel > QLORA_NOALLOC_MAX_ELEMENTS) return QLORA_ERR_WORKSPACE;
-  if (!W || !out->codes || !out->absmax_q || !out->absmax_c2 || !out->absmax_mean) return QLORA_ERR_NULL;
-  const auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-  if (!a16(W) || !a16(out->codes) || !a16(out->absmax_q) || !a16(out->absmax_c2) ||
-      !a16(out->absmax_mean))
-    return QLORA_ERR_ALIGN;
   const Nf4Tables& tabs = nf4_tables();
   if (!tabs.ok) return QLORA_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   int num_sms = 0;
-  qlora_status st = scratch_for_current_device(&scratch, &num_sms);
+  st = scratch_for_current_device(&scratch, &num_sms);
   if (st != QLORA_OK) return st;
 
   EncodeTables et;
@@ -107,14 +106,14 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const uint16_t* W, const q
   const int cap = wave < kNoAllocPartials ? wave : kNoAllocPartials;
   if (grid > cap) grid = cap;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (launch_encode(W, numel, et, out->codes, c1buf, partials, grid, s) != cudaSuccess)
+  if (counted(launch_encode(W, numel, et, out->codes, c1buf, partials, grid, s)) != cudaSuccess)
     return QLORA_ERR_CUDA;
   const int64_t ngroups = (nblocks + 255) / 256;
   int grid2 = static_cast<int>((ngroups + 7) / 8);
   if (grid2 > num_sms * 4) grid2 = num_sms * 4;
   if (grid2 < 1) grid2 = 1;
-  if (launch_double_quant(c1buf, nblocks, partials, grid, out->absmax_q, out->absmax_c2,
-                          out->absmax_mean, grid2, s) != cudaSuccess)
+  if (counted(launch_double_quant(c1buf, nblocks, partials, grid, out->absmax_q, out->absmax_c2,
+                                  out->absmax_mean, grid2, s)) != cudaSuccess)
     return QLORA_ERR_CUDA;
   return QLORA_OK;
 }

@@ -83,9 +83,11 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete.  Returns false
+// Bounded wait for the phase with the given parity to complete: gives up once
+// `limit_cycles` SM cycles have passed after the fast polls.  Returns false
 // (and sets the error flag) if it gave up; callers then stop their role.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                              long long limit_cycles) {
 #pragma unroll 1
   for (int i = 0; i < kFastPolls; ++i)
     if (mbar_try_wait(bar, parity)) return true;
@@ -94,10 +96,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
 #pragma unroll 1
     for (int i = 0; i < 256; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (clock_cycles() - t0 > kWaitLimitCycles) break;
+    if (clock_cycles() - t0 > limit_cycles) break;
   }
   if (err) atomicOr(err, kErrWaitTimeout);
   return false;
+}
+
+// The wait every pipeline in the library uses: limit kWaitLimitCycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  return mbar_wait_for(bar, parity, err, kWaitLimitCycles);
 }
 
 // ---------------------------------------------------------------- proxies

@@ -32,6 +32,11 @@
  *   - Inputs must be finite.  Non-finite weights give unspecified codes.
  *   - Thread safety: calls may be made concurrently on different streams;
  *     calls sharing a work buffer must be ordered by the caller.
+ *   - Reproducibility: NF4 codes, E4M3 constants, c2, the mean and the
+ *     dequantized weight are bit-exact and deterministic.  Results that sum
+ *     split-K partials with fp32 atomics can differ in the last bits from run
+ *     to run (the order of the additions varies): the saved X A^T, dA and dB
+ *     with more than 16 tokens, and dX with 16 tokens or fewer.
  */
 #ifndef QLORA_H_
 #define QLORA_H_
@@ -191,8 +196,10 @@ QLORA_EXPORT qlora_status qlora_read_device_errors(uint32_t* flags, int clear);
  * partial sums, 8 MiB + 16 KiB) is a fixed array inside the library that
  * every GPU loading the library holds until the process exits.
  *   - Same arguments and results as qlora_quantize_nf4_dq, bit for bit.
- *   - rows * cols above QLORA_NOALLOC_MAX_ELEMENTS: QLORA_ERR_WORKSPACE,
- *     nothing launched.  Other validation as for qlora_quantize_nf4_dq.
+ *   - Validation as for qlora_quantize_nf4_dq, in the same order; where that
+ *     entry point checks its work buffer's size, this one checks rows * cols
+ *     against QLORA_NOALLOC_MAX_ELEMENTS (QLORA_ERR_WORKSPACE above it, with
+ *     nothing launched).
  *   - The first call on a device (with that device current) looks up the
  *     array's device address; make that first call before any stream capture.
  *   - All calls share the one array: calls that can overlap on the GPU (other
@@ -201,6 +208,20 @@ QLORA_EXPORT qlora_status qlora_read_device_errors(uint32_t* flags, int clear);
  *   - Calls no cudaMalloc / cudaFree or other allocating routine.
  */
 QLORA_EXPORT qlora_status qlora_quantize_nf4_dq_noalloc(const uint16_t* W, const qlora_nf4_tensor* out,
+                                                     qlora_stream_t stream);
+
+/*
+ * Self-test of the failure path (no counterpart on the pages): launches one
+ * CTA that waits on an mbarrier nothing arrives on, with the library's bounded
+ * wait and a limit of `limit_cycles` SM cycles (0 .. 1e8) instead of the
+ * pipelines' two seconds.  No copy or MMA is in flight, so the wait gives up:
+ * the kernel sets bit 0 (wait timed out) of the device error flag that
+ * qlora_read_device_errors reads, writes 1 to *outcome (2 if the wait had
+ * completed; outcome may be NULL, else a 4-byte aligned device pointer) and
+ * returns, leaving the context usable.
+ * Errors: QLORA_ERR_SHAPE (limit out of range), QLORA_ERR_ALIGN.
+ */
+QLORA_EXPORT qlora_status qlora_selftest_bounded_wait(int64_t limit_cycles, uint32_t* outcome,
                                                      qlora_stream_t stream);
 
 /*

@@ -297,6 +297,19 @@ def linear_bwd(Wd, X, dY, A, B, s: float):
     return dX, dA, dB
 
 
+def lora_grads(X, dY, A, B, s: float):
+    """The LoRA branch's own quantities, in float64 (they do not involve W):
+    XA = X A^T [M, r], G = dY B [M, r], dA = s G^T X [r, K], dB = s dY^T XA [N, r].
+    Same formulas as linear_fwd / linear_bwd (automatone "QLoRA paper explained",
+    "How it works": the gradients land only on the LoRA adapters)."""
+    X, dY, A, B = _f64(X), _f64(dY), _f64(A), _f64(B)
+    XA = X @ A.T
+    G = dY @ B
+    dA = s * (G.T @ X)
+    dB = s * (dY.T @ XA)
+    return XA, G, dA, dB
+
+
 def linear_fwd_rows(Wd, X, A, B, s: float, rows):
     """Forward restricted to selected token rows (exactly the same formula)."""
     return linear_fwd(Wd, np.asarray(X)[rows], A, B, s)[0]

@@ -143,3 +143,53 @@ def test_linear_pointer_validation():
 def test_status_strings():
     for st in (OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_UNSUP, ERR_CUDA, ERR_WS, 12345):
         assert isinstance(qb.qlora_status_string(st), str) and qb.qlora_status_string(st)
+
+
+def test_noalloc_validates_like_the_workspace_entry_point():
+    """The allocation-free quantize runs the same descriptor checks in the same
+    order as qlora_quantize_nf4_dq, so a bad call gets the same status from
+    both; only its size limit replaces the work-buffer check."""
+    w, ws = ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000)
+    huge_cols = _tensor(rows=0, cols=(1 << 31) + 64)          # empty, but cols out of range
+    bad_bs = _tensor()
+    bad_bs.blocksize2 = 128
+    mis = _tensor()
+    mis.absmax_mean = mis.absmax_mean + 8
+    nul = _tensor()
+    nul.absmax_q = None
+    cases = [(w, huge_cols, ERR_SHAPE), (w, bad_bs, ERR_UNSUP), (w, mis, ERR_ALIGN), (w, nul, ERR_NULL),
+             (None, _tensor(), ERR_NULL), (ctypes.c_void_p(0x20004), _tensor(), ERR_ALIGN)]
+    for wp, t, expect in cases:
+        a = lib.qlora_quantize_nf4_dq(wp, ctypes.byref(t), ws, 1 << 40, None)
+        b = lib.qlora_quantize_nf4_dq_noalloc(wp, ctypes.byref(t), None)
+        assert a == b == expect, (a, b, expect)
+    assert lib.qlora_quantize_nf4_dq_noalloc(w, None, None) == ERR_NULL
+    big = _tensor(rows=2, cols=qb.NOALLOC_MAX_ELEMENTS // 2 + 64)
+    assert lib.qlora_quantize_nf4_dq_noalloc(w, ctypes.byref(big), None) == ERR_WS
+
+
+def test_python_wrapper_refuses_a_destination_of_another_shape():
+    """The C entry points read out.rows * out.cols weights from W; the binding
+    refuses a destination that describes more (or fewer) weights than W holds,
+    or that lives on another device, before calling the library."""
+    import torch
+    w = torch.zeros(64, 128, dtype=torch.bfloat16)
+    cpu = torch.device("cpu")
+    good = qb.NF4Tensor(codes=torch.zeros(4096, dtype=torch.uint8), absmax_q=torch.zeros(128, dtype=torch.uint8),
+                        absmax_c2=torch.zeros(4), absmax_mean=torch.zeros(4), rows=64, cols=128)
+    qb._check_out_matches(w, good)
+    bigger = qb.NF4Tensor(codes=good.codes, absmax_q=good.absmax_q, absmax_c2=good.absmax_c2,
+                          absmax_mean=good.absmax_mean, rows=128, cols=128)
+    with pytest.raises(ValueError, match="describes"):
+        qb._check_out_matches(w, bigger)
+    meta = qb.NF4Tensor(codes=torch.empty(4096, dtype=torch.uint8, device="meta"), absmax_q=good.absmax_q,
+                        absmax_c2=good.absmax_c2, absmax_mean=good.absmax_mean, rows=64, cols=128)
+    assert meta.codes.device != cpu
+    with pytest.raises(ValueError, match="codes"):
+        qb._check_out_matches(w, meta)
+
+
+def test_selftest_rejects_limits_out_of_range():
+    assert lib.qlora_selftest_bounded_wait(-1, None, None) == ERR_SHAPE
+    assert lib.qlora_selftest_bounded_wait(100000001, None, None) == ERR_SHAPE
+    assert lib.qlora_selftest_bounded_wait(1000, ctypes.c_void_p(0x40002), None) == ERR_ALIGN

@@ -49,6 +49,32 @@ def test_forward_and_backward_match_autograd():
     assert np.max(np.abs(dB - Bt.grad.numpy())) <= 1e-12 * rms(dB)
 
 
+def test_lora_grads_match_autograd():
+    """oracle.lora_grads (X A^T, dY B, dA, dB: what the GPU parity tests compare
+    against at full size) against torch float64 autograd of the LoRA branch
+    alone, and its intermediates against the hidden activations autograd saw."""
+    _, X, A, B, dY = _case(m=24, n=40, k=128, r=16, proj=4)
+    s = 0.25
+    XA, G, dA, dB = oracle.lora_grads(X, dY, A, B, s)
+    Xt = torch.tensor(X, dtype=torch.float64)
+    At = torch.tensor(A, dtype=torch.float64, requires_grad=True)
+    Bt = torch.tensor(B, dtype=torch.float64, requires_grad=True)
+    H = torch.nn.functional.linear(Xt, At)            # X A^T
+    H.retain_grad()
+    Yl = s * torch.nn.functional.linear(H, Bt)
+    Yl.backward(torch.tensor(dY, dtype=torch.float64))
+    rms = lambda a: float(np.sqrt(np.mean(np.square(a))))
+    assert np.max(np.abs(XA - H.detach().numpy())) <= 1e-12 * rms(XA)
+    # dL/dH = s dY B = s G
+    assert np.max(np.abs(s * G - H.grad.numpy())) <= 1e-12 * rms(G)
+    assert np.max(np.abs(dA - At.grad.numpy())) <= 1e-12 * rms(dA)
+    assert np.max(np.abs(dB - Bt.grad.numpy())) <= 1e-12 * rms(dB)
+    # the same quantities as the full layer's backward (W only adds to dX)
+    Wd = np.zeros((40, 128), np.float32)
+    _, dA2, dB2 = oracle.linear_bwd(Wd, X, dY, A, B, s)
+    assert np.array_equal(dA, dA2) and np.array_equal(dB, dB2)
+
+
 def test_zero_lora_reduces_to_plain_matmul():
     Wd, X, A, B, dY = _case(m=8, n=32, k=128, r=4, proj=1)
     Y0, _ = oracle.linear_fwd(Wd, X, A, np.zeros_like(B), 2.0)

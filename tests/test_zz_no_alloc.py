@@ -52,8 +52,11 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls(qb):
             t.fill_(0xA5)                       # poison: every byte must be rewritten
         got.absmax_c2.fill_(float("nan"))
         c = got.c_struct()
+        launches0 = qb.qlora_kernel_launches()
         st = qb._lib.qlora_quantize_nf4_dq_noalloc(ctypes.c_void_p(w.data_ptr()), ctypes.byref(c), stream)
         assert st == 0, qb.qlora_status_string(st)
+        # the encoder and the double quantization, counted like every launch
+        assert qb.qlora_kernel_launches() - launches0 == 2
         torch.cuda.synchronize()
         assert qb.qlora_read_device_errors() == 0
         a = _stored(ref, sz["codes"], sz["absmax_q"], ngroups)
