@@ -392,7 +392,41 @@ def secondary(qb, torch, device, peaks):
             out[f"gemv_{n}x{k}_m{m}"] = {"us": round(t * 1e6, 2), "GB/s": round(gbs, 1),
                                          "frac_hbm": round(gbs / hbm, 4), "bytes": byts}
             del g
+        if n > k:
+            # several adapters over the same weight, one per group of tokens (16 tokens)
+            for n_ad in (4, 16):
+                m = 16
+                X = workloads.activations(m, k, 31).to(device)
+                Y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+                A_st = torch.stack([workloads.lora_a(64, k, 60 + a) for a in range(n_ad)]).to(device)
+                B_st = torch.stack([workloads.lora_b(n, 64, 60 + a) for a in range(n_ad)]).to(device)
+                idx = (torch.arange(m, dtype=torch.int32) % n_ad).to(device)
+                wsz = torch.empty(qb.qlora_linear_workspace_size(n, k, m, 64)[0], dtype=torch.uint8, device=device)
+                call = lambda j: qb.qlora_linear_fwd_multi(wsets[j % 2], X, A_st, B_st, idx, 0.25, save_xa=False,
+                                                           Y=Y, workspace=wsz)
+                t = graph_time(torch, lambda: [call(j) for j in range(2)], 10, 5) / 2
+                byts = (szg["codes"] + szg["absmax_q"] + szg["absmax_c2"] + 4 + n_ad * (A.numel() + B.numel()) * 2
+                        + m * k * 2 + m * n * 2)
+                gbs = byts / t / 1e9
+                out[f"gemv_multi_{n}x{k}_m{m}_adapters{n_ad}"] = {"us": round(t * 1e6, 2), "GB/s": round(gbs, 1),
+                                                                   "frac_hbm": round(gbs / hbm, 4), "bytes": byts}
         del wsets
+    # the stored form without double quantization: fp32 block constants (0.5 bits
+    # per weight); 4 weight sets rotated (4 x 42 MB > L2), as for the DQ form
+    wp = [workloads.weight((4096, 4096), proj=j, outliers=True).to(device) for j in range(4)]
+    qp = [qb.qlora_quantize_nf4_dq(x, double_quant=False) for x in wp]
+    outp = [torch.empty(4096, 4096, dtype=torch.bfloat16, device=device) for _ in range(4)]
+    szp = qb.qlora_nf4_sizes(4096, 4096, double_quant=False)
+    wsp = torch.empty(szp["workspace"], dtype=torch.uint8, device=device)
+    pbytes = 4096 * 4096 * 2 + szp["codes"] + szp["absmax_q"]
+    for name, fn in (("encode_nodq_4096x4096",
+                      lambda: [qb.qlora_quantize_nf4_dq(wp[j], out=qp[j], workspace=wsp) for j in range(4)]),
+                     ("dequant_nodq_4096x4096", lambda: [qb.qlora_dequantize(qp[j], out=outp[j]) for j in range(4)])):
+        t = graph_time(torch, fn, 5, 2) / 4
+        out[name] = {"us": round(t * 1e6, 2), "GB/s": round(pbytes / t / 1e9, 1),
+                     "frac_hbm": round(pbytes / t / 1e9 / hbm, 4), "bytes": pbytes}
+    del wp, qp, outp
+    out["bits_per_param_nodq"] = round(8 * (szp["codes"] + szp["absmax_q"]) / (4096 * 4096), 6)
     return out
 
 

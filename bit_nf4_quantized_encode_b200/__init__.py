@@ -10,6 +10,7 @@ Entry points (same names as the C ABI):
     qlora_quantize_nf4_dq(W)                          -> NF4Tensor
     qlora_dequantize(qt)                              -> bf16 [rows, cols]
     qlora_linear_fwd(qt, X, A, B, s, save_xa=True)    -> (Y bf16, XA fp32 or None)
+    qlora_linear_fwd_multi(qt, X, A_stack, B_stack, adapter_idx, s) -> (Y, XA): one adapter per token
     qlora_linear_bwd(qt, X, dY, A, B, s, XA=None, need_dx=True) -> (dX bf16 or None, dA fp32, dB fp32)
     qlora_get_codebook()                              -> 16 float levels
 """
@@ -37,7 +38,12 @@ class _Nf4TensorC(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("absmax_q", ctypes.c_void_p),
                 ("absmax_c2", ctypes.c_void_p), ("absmax_mean", ctypes.c_void_p),
                 ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
-                ("blocksize", ctypes.c_int32), ("blocksize2", ctypes.c_int32)]
+                ("blocksize", ctypes.c_int32), ("blocksize2", ctypes.c_int32),
+                ("absmax", ctypes.c_void_p), ("quant_type", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+# The 4-bit data types (qlora_quant_type): NF4 and the two it is compared with.
+QUANT_TYPES = {"nf4": 0, "fp4": 1, "int4": 2}
 
 
 _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
@@ -48,6 +54,8 @@ _lib.qlora_status_string.argtypes = [ctypes.c_int]
 _lib.qlora_status_string.restype = ctypes.c_char_p
 _lib.qlora_get_codebook.argtypes = [ctypes.POINTER(ctypes.c_float)]
 _lib.qlora_get_codebook.restype = None
+_lib.qlora_get_levels.argtypes = [_i32, ctypes.POINTER(ctypes.c_float)]
+_lib.qlora_get_levels.restype = ctypes.c_int
 _lib.qlora_nf4_sizes.argtypes = [_i64, _i64, _i32, _i32, _szp, _szp, _szp, _szp]
 _lib.qlora_nf4_sizes.restype = ctypes.c_int
 _lib.qlora_quantize_nf4_dq.argtypes = [_vp, _T, _vp, _sz, _vp]
@@ -59,6 +67,9 @@ _lib.qlora_linear_workspace_size.restype = ctypes.c_int
 _lib.qlora_linear_fwd.argtypes = [_T, _vp, _i64, _vp, _vp, _i32, ctypes.c_float, _vp, _vp, _vp,
                                   _sz, _vp]
 _lib.qlora_linear_fwd.restype = ctypes.c_int
+_lib.qlora_linear_fwd_multi.argtypes = [_T, _vp, _i64, _vp, _vp, _i32, _vp, _i32, ctypes.c_float, _vp, _vp,
+                                        _vp, _sz, _vp]
+_lib.qlora_linear_fwd_multi.restype = ctypes.c_int
 _lib.qlora_linear_bwd.argtypes = [_T, _vp, _vp, _i64, _vp, _vp, _i32, ctypes.c_float, _vp, _vp,
                                   _vp, _vp, _vp, _sz, _vp]
 _lib.qlora_linear_bwd.restype = ctypes.c_int
@@ -73,8 +84,8 @@ _lib.qlora_time_next_gemm.restype = ctypes.c_int
 _lib.qlora_selftest_bounded_wait.argtypes = [_i64, _vp, _vp]
 _lib.qlora_selftest_bounded_wait.restype = ctypes.c_int
 
-EXPORTED = ["qlora_status_string", "qlora_get_codebook", "qlora_nf4_sizes", "qlora_quantize_nf4_dq",
-            "qlora_dequantize", "qlora_linear_workspace_size", "qlora_linear_fwd",
+EXPORTED = ["qlora_status_string", "qlora_get_codebook", "qlora_get_levels", "qlora_nf4_sizes", "qlora_quantize_nf4_dq",
+            "qlora_dequantize", "qlora_linear_workspace_size", "qlora_linear_fwd", "qlora_linear_fwd_multi",
             "qlora_linear_bwd", "qlora_read_device_errors", "qlora_kernel_launches",
             "qlora_time_next_gemm", "qlora_quantize_nf4_dq_noalloc", "qlora_selftest_bounded_wait"]
 
@@ -109,26 +120,39 @@ def _need_bf16_cuda(name: str, t: torch.Tensor):
 
 @dataclass
 class NF4Tensor:
-    """A quantized weight: packed codes, E4M3 block constants, c2 per group, mean."""
-    codes: torch.Tensor        # uint8 [ceil(rows*cols/2)]
-    absmax_q: torch.Tensor     # uint8 [ceil(rows*cols/64)]
-    absmax_c2: torch.Tensor    # float32 [ceil(nblocks/256)]
-    absmax_mean: torch.Tensor  # float32 [1]
+    """A quantized weight: packed 4-bit codes and its block constants, stored
+    either double-quantized (E4M3 codes, c2 per group, mean) or as fp32 absmax
+    per block (`absmax`, no double quantization)."""
+    codes: torch.Tensor                     # uint8 [ceil(rows*cols/2)]
+    absmax_q: torch.Tensor | None           # uint8 [ceil(rows*cols/64)] (double quantization)
+    absmax_c2: torch.Tensor | None          # float32 [ceil(nblocks/256)] (double quantization)
+    absmax_mean: torch.Tensor | None        # float32 [1] (double quantization)
     rows: int
     cols: int
+    absmax: torch.Tensor | None = None      # float32 [nblocks] (no double quantization)
+    quant_type: str = "nf4"                 # "nf4", "fp4" or "int4"
+
+    @property
+    def double_quant(self) -> bool:
+        return self.absmax is None
 
     def c_struct(self) -> _Nf4TensorC:
-        return _Nf4TensorC(self.codes.data_ptr(), self.absmax_q.data_ptr(),
-                           self.absmax_c2.data_ptr(), self.absmax_mean.data_ptr(),
-                           self.rows, self.cols, BLOCKSIZE, BLOCKSIZE2)
+        p = lambda t: 0 if t is None else t.data_ptr()
+        return _Nf4TensorC(self.codes.data_ptr(), p(self.absmax_q), p(self.absmax_c2), p(self.absmax_mean),
+                           self.rows, self.cols, BLOCKSIZE, BLOCKSIZE2 if self.double_quant else 0,
+                           p(self.absmax), QUANT_TYPES[self.quant_type], 0)
+
+    def buffers(self) -> dict:
+        return {n: t for n, t in (("codes", self.codes), ("absmax_q", self.absmax_q),
+                                  ("absmax_c2", self.absmax_c2), ("absmax_mean", self.absmax_mean),
+                                  ("absmax", self.absmax)) if t is not None}
 
     @property
     def device(self):
         return self.codes.device
 
     def nbytes(self) -> int:
-        return sum(t.numel() * t.element_size() for t in
-                   (self.codes, self.absmax_q, self.absmax_c2, self.absmax_mean))
+        return sum(t.numel() * t.element_size() for t in self.buffers().values())
 
 
 def qlora_status_string(status: int) -> str:
@@ -141,22 +165,37 @@ def qlora_get_codebook() -> list:
     return list(out)
 
 
-def qlora_nf4_sizes(rows: int, cols: int) -> dict:
+def qlora_get_levels(quant_type: str = "nf4") -> list:
+    """The 16 levels of a 4-bit type ("nf4", "fp4" or "int4")."""
+    out = (ctypes.c_float * 16)()
+    _check(_lib.qlora_get_levels(QUANT_TYPES[quant_type], out), "qlora_get_levels")
+    return list(out)
+
+
+def qlora_nf4_sizes(rows: int, cols: int, double_quant: bool = True) -> dict:
+    """Buffer sizes in bytes; without double quantization 'absmax_q' is the
+    size of the fp32 absmax array and 'absmax_c2' is 0."""
     v = [ctypes.c_size_t() for _ in range(4)]
-    _check(_lib.qlora_nf4_sizes(rows, cols, BLOCKSIZE, BLOCKSIZE2, *[ctypes.byref(x) for x in v]),
-           "qlora_nf4_sizes")
+    _check(_lib.qlora_nf4_sizes(rows, cols, BLOCKSIZE, BLOCKSIZE2 if double_quant else 0,
+                                *[ctypes.byref(x) for x in v]), "qlora_nf4_sizes")
     return dict(codes=v[0].value, absmax_q=v[1].value, absmax_c2=v[2].value, workspace=v[3].value)
 
 
-def empty_nf4(rows: int, cols: int, device) -> NF4Tensor:
-    sz = qlora_nf4_sizes(rows, cols)
+def empty_nf4(rows: int, cols: int, device, quant_type: str = "nf4", double_quant: bool = True) -> NF4Tensor:
+    if quant_type not in QUANT_TYPES:
+        raise ValueError(f"quant_type must be one of {sorted(QUANT_TYPES)}")
+    sz = qlora_nf4_sizes(rows, cols, double_quant)
     # round each buffer up to 16 bytes so every pointer the library sees is aligned
     def buf(n, dtype, esize):
         return torch.empty(max(1, (n + 15) // 16 * 16 // esize), dtype=dtype, device=device)
-    return NF4Tensor(codes=buf(sz["codes"], torch.uint8, 1), absmax_q=buf(sz["absmax_q"], torch.uint8, 1),
+    codes = buf(sz["codes"], torch.uint8, 1)
+    if not double_quant:
+        return NF4Tensor(codes=codes, absmax_q=None, absmax_c2=None, absmax_mean=None, rows=rows, cols=cols,
+                         absmax=buf(sz["absmax_q"], torch.float32, 4), quant_type=quant_type)
+    return NF4Tensor(codes=codes, absmax_q=buf(sz["absmax_q"], torch.uint8, 1),
                      absmax_c2=buf(sz["absmax_c2"], torch.float32, 4),
                      absmax_mean=torch.empty(4, dtype=torch.float32, device=device),
-                     rows=rows, cols=cols)
+                     rows=rows, cols=cols, quant_type=quant_type)
 
 
 def _check_out_matches(W: torch.Tensor, out: NF4Tensor):
@@ -164,21 +203,22 @@ def _check_out_matches(W: torch.Tensor, out: NF4Tensor):
     weights from W: refuse a destination that describes another tensor."""
     if out.rows * out.cols != W.numel():
         raise ValueError(f"out describes {out.rows}x{out.cols} weights, W has {W.numel()}")
-    for name, t in (("codes", out.codes), ("absmax_q", out.absmax_q), ("absmax_c2", out.absmax_c2),
-                    ("absmax_mean", out.absmax_mean)):
+    for name, t in out.buffers().items():
         if t.device != W.device:
             raise ValueError(f"out.{name} is on {t.device}, W on {W.device}")
 
 
 def qlora_quantize_nf4_dq(W: torch.Tensor, out: NF4Tensor | None = None,
-                          workspace: torch.Tensor | None = None) -> NF4Tensor:
-    """Blockwise NF4 encode + double quantization of a bf16 [rows, cols] weight."""
+                          workspace: torch.Tensor | None = None, quant_type: str = "nf4",
+                          double_quant: bool = True) -> NF4Tensor:
+    """Blockwise 4-bit encode (NF4 by default) + double quantization of a bf16
+    [rows, cols] weight; `out`, when given, fixes the type and the form."""
     _need_bf16_cuda("W", W)
     rows, cols = (W.shape[0], W.shape[1]) if W.dim() == 2 else (1, W.numel())
     if out is None:
-        out = empty_nf4(rows, cols, W.device)
+        out = empty_nf4(rows, cols, W.device, quant_type, double_quant)
     _check_out_matches(W, out)
-    need = qlora_nf4_sizes(rows, cols)["workspace"]
+    need = qlora_nf4_sizes(out.rows, out.cols, out.double_quant)["workspace"]
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
     c = out.c_struct()
@@ -232,6 +272,37 @@ def qlora_linear_fwd(qt: NF4Tensor, X: torch.Tensor, A: torch.Tensor, B: torch.T
     _check(_lib.qlora_linear_fwd(ctypes.byref(c), _ptr(X), m, _ptr(A), _ptr(B), r, float(s), _ptr(Y),
                                  _ptr(XA if save_xa else None), _ptr(workspace), workspace.numel(),
                                  _stream(X.device)), "qlora_linear_fwd")
+    return Y, (XA if save_xa else None)
+
+
+def qlora_linear_fwd_multi(qt: NF4Tensor, X: torch.Tensor, A_stack: torch.Tensor, B_stack: torch.Tensor,
+                           adapter_idx: torch.Tensor, s: float, save_xa: bool = True,
+                           Y: torch.Tensor | None = None, XA: torch.Tensor | None = None,
+                           workspace: torch.Tensor | None = None):
+    """Decode-shaped forward (M <= 16) with one adapter per token:
+    Y[t] = X[t] deq(W)^T + s (X[t] A_a^T) B_a^T with a = adapter_idx[t]
+    (int32 on the device; negative = no adapter).  A_stack [n, r, cols] and
+    B_stack [n, rows, r] bf16.  Returns (Y bf16, XA fp32 or None)."""
+    for n, t in (("X", X), ("A_stack", A_stack), ("B_stack", B_stack)):
+        _need_bf16_cuda(n, t)
+    if not (adapter_idx.is_cuda and adapter_idx.dtype == torch.int32 and adapter_idx.is_contiguous()
+            and adapter_idx.numel() == X.shape[0]):
+        raise ValueError("adapter_idx must be a contiguous int32 CUDA tensor with one entry per token")
+    if A_stack.dim() != 3 or B_stack.dim() != 3 or A_stack.shape[0] != B_stack.shape[0]:
+        raise ValueError("A_stack [n, r, cols] and B_stack [n, rows, r] must hold the same adapters")
+    m, n_ad, r = X.shape[0], A_stack.shape[0], A_stack.shape[1]
+    if Y is None:
+        Y = torch.empty(m, qt.rows, dtype=torch.bfloat16, device=X.device)
+    if save_xa and XA is None:
+        XA = torch.empty(m, r, dtype=torch.float32, device=X.device)
+    if workspace is None:
+        workspace = torch.empty(qlora_linear_workspace_size(qt.rows, qt.cols, m, r)[0],
+                                dtype=torch.uint8, device=X.device)
+    c = qt.c_struct()
+    _check(_lib.qlora_linear_fwd_multi(ctypes.byref(c), _ptr(X), m, _ptr(A_stack), _ptr(B_stack), n_ad,
+                                       _ptr(adapter_idx), r, float(s), _ptr(Y), _ptr(XA if save_xa else None),
+                                       _ptr(workspace), workspace.numel(), _stream(X.device)),
+           "qlora_linear_fwd_multi")
     return Y, (XA if save_xa else None)
 
 

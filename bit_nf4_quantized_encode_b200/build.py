@@ -14,8 +14,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libqlora.so")
-SOURCES = ["api.cu", "codec.cu", "gemm.cu", "gemv.cu", "noalloc.cu", "selftest.cu", "nf4_tables.cpp"]
-HEADERS = ["codec.h", "gemm.h", "gemv.h", "internal.h", "nf4_device.cuh", "nf4_tables.h", "sm100_ptx.cuh"]
+SOURCES = ["api.cu", "codec.cu", "gemm.cu", "gemv.cu", "lora.cu", "noalloc.cu", "selftest.cu", "nf4_tables.cpp"]
+HEADERS = ["codec.h", "gemm.h", "gemv.h", "internal.h", "lora.h", "nf4_device.cuh", "nf4_tables.h", "sm100_ptx.cuh"]
 
 
 def _newest_input() -> float:

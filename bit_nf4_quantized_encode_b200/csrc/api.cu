@@ -16,6 +16,7 @@
 #include "gemm.h"
 #include "gemv.h"
 #include "internal.h"
+#include "lora.h"
 #include "nf4_tables.h"
 #include "qlora.h"
 
@@ -143,12 +144,15 @@ int balanced_splits(int tiles, int ksteps, int sms) {
   return best;
 }
 
-CodebookParam codebook_param() {
+CodebookParam codebook_param(int type) {
   CodebookParam cb;
-  const Nf4Tables& t = nf4_tables();
+  const Nf4Tables& t = level_tables(type);
   for (int i = 0; i < 16; ++i) cb.level[i] = t.level[i];
   return cb;
 }
+
+// fp32 block constants of a weight stored without double quantization, else NULL
+const float* plain_absmax(const qlora_nf4_tensor* t) { return t->blocksize2 == 0 ? t->absmax : nullptr; }
 
 qlora_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
 
@@ -177,10 +181,32 @@ qlora_status check_linear(const qlora_nf4_tensor* W, int64_t M, int32_t r, Linea
 
 // Work buffer layout: fp32 accumulators first (one memset clears them all),
 // then bf16 staging.  Offsets in bytes, each 256-aligned.
-struct FwdLayout {
-  size_t xa_acc, cnt, slots, fp32_end, sxa, xa_slices, total;
+// Splits of the rank-r contractions are sized for up to this many SMs, so a
+// work buffer sized without a device fits any device's launch.
+constexpr int kSizingSms = 256;
+constexpr int kMaxRankSplits = 32;
+
+// One rank-r contraction's tiling: tiles of 128 rows x 64 columns, K splits.
+struct RankPlan {
+  int m_tiles, n_tiles, ksteps, splits;
+  int tiles() const { return m_tiles * n_tiles; }
 };
-FwdLayout fwd_layout(const LinearShape& s) {
+RankPlan rank_plan(int64_t mdim, int64_t contraction, int lora_steps, int sms_tiles_total, int num_sms) {
+  RankPlan p;
+  p.m_tiles = static_cast<int>((mdim + 127) / 128);
+  p.n_tiles = lora_steps;
+  p.ksteps = static_cast<int>((contraction + 63) / 64);
+  p.splits = rank_splits(sms_tiles_total, p.ksteps, num_sms, kMaxRankSplits);
+  return p;
+}
+
+// Work buffer layout: the region cleared by one memset first (counters, and
+// the decode backward's split-K dX accumulator), then the rest.  Offsets in
+// bytes, each 256-aligned.
+struct FwdLayout {
+  size_t cnt, slots, xa_slices, sxa, rank_cnt, rank_slots, clear_end, total;
+};
+FwdLayout fwd_layout(const LinearShape& s, int num_sms = kSizingSms) {
   FwdLayout l{};
   size_t o = 0;
   if (s.decode) {        // k_xa_zero + k_gemv: tile counters, partial slots, X A^T slices
@@ -189,57 +215,119 @@ FwdLayout fwd_layout(const LinearShape& s) {
     l.cnt = o;      o = round_up(o + m_tiles * 8 * 4, 256);
     l.slots = o;    o = round_up(o + size_t(gemv_slot_floats(int64_t(m_tiles), int64_t(steps))) * 4, 256);
     l.xa_slices = o; o = round_up(o + size_t(kMaxXaSplits) * 16 * s.rpad * 4, 256);
-    l.fp32_end = 0;
+    l.clear_end = 0;
     l.total = o;
     return l;
   }
-  l.xa_acc = o; o = round_up(o + size_t(s.m) * s.rpad * 4, 256);
-  l.fp32_end = o;
+  // k_rank (X A^T -> bf16(s X A^T)) then the fused dequant-GEMM
+  const RankPlan xa = rank_plan(s.m, s.cols, s.lora_steps,
+                                int((s.m + 127) / 128) * s.lora_steps, num_sms);
+  l.rank_cnt = o;   o = round_up(o + size_t(xa.tiles()) * 4, 256);
+  l.clear_end = o;
+  l.rank_slots = o; o = round_up(o + rank_slot_bytes(xa.tiles(), xa.splits), 256);
+  l.sxa = o;        o = round_up(o + size_t(s.m) * s.rpad * 2, 256);
+  l.total = o;
+  return l;
+}
+
+// Backward: launch 1 = dY B (and X A^T when it is not supplied), launch 2 =
+// the fused dX, launch 3 = dY^T (s X A^T) and X^T (s dY B) (more than 16
+// tokens; with fewer, k_small_grads from the fp32 G and X A^T).
+struct BwdLayout {
+  size_t cnt1, cnt2, dx_acc, clear_end, slots1, slots2, g, xa, sg, sxa, total;
+  RankPlan g_plan, xa_plan, db_plan, da_plan;
+};
+BwdLayout bwd_layout(const LinearShape& s, int num_sms = kSizingSms) {
+  BwdLayout l{};
+  // launch 1 is planned for both problems whether or not X A^T is recomputed,
+  // so that the layout does not depend on the call
+  const int t1 = 2 * int((s.m + 127) / 128) * s.lora_steps;
+  l.g_plan = rank_plan(s.m, s.rows, s.lora_steps, t1, num_sms);
+  l.xa_plan = rank_plan(s.m, s.cols, s.lora_steps, t1, num_sms);
+  const int t2 = int((s.rows + 127) / 128 + (s.cols + 127) / 128) * s.lora_steps;
+  l.db_plan = rank_plan(s.rows, s.m, s.lora_steps, t2, num_sms);
+  l.da_plan = rank_plan(s.cols, s.m, s.lora_steps, t2, num_sms);
+  size_t o = 0;
+  l.cnt1 = o;   o = round_up(o + size_t(l.g_plan.tiles() + l.xa_plan.tiles()) * 4, 256);
+  l.cnt2 = o;   o = round_up(o + size_t(l.db_plan.tiles() + l.da_plan.tiles()) * 4, 256);
+  l.dx_acc = o; if (s.decode) o = round_up(o + size_t(s.m) * s.cols * 4, 256);
+  l.clear_end = o;
+  l.slots1 = o; o = round_up(o + rank_slot_bytes(l.g_plan.tiles(), l.g_plan.splits) +
+                             rank_slot_bytes(l.xa_plan.tiles(), l.xa_plan.splits), 256);
+  l.slots2 = o; if (!s.decode) o = round_up(o + rank_slot_bytes(l.db_plan.tiles(), l.db_plan.splits) +
+                                            rank_slot_bytes(l.da_plan.tiles(), l.da_plan.splits), 256);
+  l.g = o;      if (s.decode) o = round_up(o + size_t(s.m) * s.rpad * 4, 256);
+  l.xa = o;     if (s.decode) o = round_up(o + size_t(s.m) * s.rpad * 4, 256);
+  l.sg = o;     o = round_up(o + size_t(s.m) * s.rpad * 2, 256);
   l.sxa = o;    o = round_up(o + size_t(s.m) * s.rpad * 2, 256);
   l.total = o;
   return l;
 }
 
-struct BwdLayout {
-  size_t g_acc, xa_acc, dx_acc, da_acc, db_acc, fp32_end, sg, xa, total;
-};
-BwdLayout bwd_layout(const LinearShape& s) {
-  BwdLayout l{};
-  size_t o = 0;
-  l.g_acc = o;  o = round_up(o + size_t(s.m) * s.rpad * 4, 256);
-  l.xa_acc = o; o = round_up(o + size_t(s.m) * s.rpad * 4, 256);
-  l.dx_acc = o; if (s.decode) o = round_up(o + size_t(s.m) * s.cols * 4, 256);
-  l.da_acc = o; o = round_up(o + size_t(s.cols) * s.rpad * 4, 256);
-  l.db_acc = o; o = round_up(o + size_t(s.rows) * s.rpad * 4, 256);
-  l.fp32_end = o;
-  l.sg = o;     o = round_up(o + size_t(s.m) * s.rpad * 2, 256);
-  l.xa = o;     o = round_up(o + size_t(s.m) * s.rpad * 2, 256);
-  l.total = o;
-  return l;
-}
-
 int choose_splits(int tiles, int ksteps, int num_sms) {
-  int s = (4 * num_sms + tiles - 1) / tiles;
-  if (s > ksteps) s = ksteps;
-  if (s < 1) s = 1;
-  return s;
+  int sp = (4 * num_sms + tiles - 1) / tiles;
+  if (sp > ksteps) sp = ksteps;
+  if (sp < 1) sp = 1;
+  return sp;
 }
 
-// D[mdim, ndim] (+)= A B^T over kdim; A and B as tensor maps; fp32 acc.
-qlora_status run_skinny(bool a_mn, bool b_mn, const CUtensorMap& am, const CUtensorMap& bm,
-                        int64_t mdim, int64_t ndim, int64_t kdim, float* acc, int64_t ld_acc,
-                        const DeviceInfo& d, cudaStream_t stream) {
-  SkinnyArgs sa{};
-  sa.mdim = mdim;
-  sa.ndim = ndim;
-  sa.ksteps = static_cast<int>((kdim + 63) / 64);
-  sa.m_tiles = static_cast<int>((mdim + 127) / 128);
-  sa.n_tiles = static_cast<int>((ndim + 63) / 64);
-  sa.splits = choose_splits(sa.m_tiles * sa.n_tiles, sa.ksteps, d.num_sms);
-  sa.acc = acc;
-  sa.ld_acc = ld_acc;
-  sa.err = d.err;
-  return cuda_status(counted(launch_skinny(a_mn, b_mn, sa, am, bm, d.num_sms, stream)));
+// One rank-r problem of a k_rank launch.
+RankProblem rank_problem(const RankPlan& pl, int64_t mdim, int64_t ndim, bool a_mn, bool b_mn, int unit_begin,
+                         float* slots, uint32_t* counters) {
+  RankProblem p{};
+  p.mdim = mdim;
+  p.ndim = ndim;
+  p.ksteps = pl.ksteps;
+  p.m_tiles = pl.m_tiles;
+  p.n_tiles = pl.n_tiles;
+  p.splits = pl.splits;
+  p.unit_begin = unit_begin;
+  p.a_mn = a_mn ? 1 : 0;
+  p.b_mn = b_mn ? 1 : 0;
+  p.slots = slots;
+  p.counters = counters;
+  return p;
+}
+
+// Decode-shaped forward (M <= 16): X A^T slices and the zeroed tile counters
+// (k_xa_zero), then one pass over the packed weight that also writes Y
+// (k_gemv, the programmatic dependent of k_xa_zero).  With adapter_idx each
+// token uses its own adapter of the stacks A [n_adapters][r, cols] and
+// B [n_adapters][rows, r].
+qlora_status run_decode_fwd(const qlora_nf4_tensor* W, const uint16_t* X, const LinearShape& sh,
+                            const uint16_t* A, const uint16_t* B, const int32_t* adapter_idx, int n_adapters,
+                            float s, uint16_t* Y, float* XA_out, uint8_t* ws, const FwdLayout& L,
+                            const DeviceInfo& d, cudaStream_t cs) {
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(ws + L.cnt);
+  const int m_tiles = static_cast<int>((sh.rows + gemv_tile_rows() - 1) / gemv_tile_rows());
+  float* xa_slices = reinterpret_cast<float*>(ws + L.xa_slices);
+  const int xa_splits = xa_splits_for(sh.r, sh.cols);
+  if (counted(launch_xa_zero(X, A, sh.m, sh.cols, sh.r, xa_slices, sh.rpad, xa_splits,
+                             reinterpret_cast<float*>(cnt), static_cast<int64_t>(m_tiles) * 8, adapter_idx,
+                             n_adapters, static_cast<int64_t>(sh.r) * sh.cols, d.err, cs)) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  CUtensorMap c_map, x_act;
+  if (!make_map_u8(&c_map, W->codes, sh.cols / 2, sh.rows, sh.cols / 2, 128, gemv_tile_rows(),
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&x_act, X, sh.cols, sh.m, sh.cols * 2, static_cast<uint32_t>(sh.m)))
+    return QLORA_ERR_CUDA;
+  GemvArgs ga{};
+  ga.qabs = W->absmax_q; ga.c2 = W->absmax_c2; ga.mean = W->absmax_mean;
+  ga.absf = plain_absmax(W);
+  ga.nw = sh.rows; ga.kw = sh.cols; ga.m = sh.m;
+  ga.slots = reinterpret_cast<float*>(ws + L.slots);
+  ga.cnt = cnt;
+  ga.xa_part = xa_slices; ga.ld_xa = sh.rpad; ga.r = sh.r; ga.lora_steps = sh.lora_steps;
+  ga.xa_splits = xa_splits;
+  ga.s = s; ga.lora_b = B; ga.y = Y; ga.xa_out = XA_out;
+  ga.adapter_idx = adapter_idx; ga.n_adapters = n_adapters; ga.b_stride = sh.rows * sh.r;
+  ga.m_tiles = m_tiles;
+  ga.steps = static_cast<int>((sh.cols / 64 + 3) / 4);
+  const CodebookParam cbp = codebook_param(W->quant_type);
+  for (int i = 0; i < 16; ++i) ga.level[i] = cbp.level[i];
+  ga.err = d.err;
+  if (counted(launch_gemv(ga, c_map, x_act, d.num_sms, cs)) != cudaSuccess) return QLORA_ERR_CUDA;
+  return QLORA_OK;
 }
 
 }  // namespace
@@ -252,13 +340,36 @@ cudaError_t counted(cudaError_t e, int n) {
 qlora_status check_tensor(const qlora_nf4_tensor* t) {
   if (!t) return QLORA_ERR_NULL;
   if (t->rows < 0 || t->cols < 0 || t->rows > kMaxDim || t->cols > kMaxDim) return QLORA_ERR_SHAPE;
-  if (t->blocksize != kBlock || t->blocksize2 != kBlock2) return QLORA_ERR_UNSUPPORTED;
+  if (t->blocksize != kBlock || (t->blocksize2 != kBlock2 && t->blocksize2 != 0)) return QLORA_ERR_UNSUPPORTED;
+  if (t->quant_type < 0 || t->quant_type >= kNumTypes || t->reserved != 0) return QLORA_ERR_UNSUPPORTED;
   if (t->rows * t->cols == 0) return QLORA_OK;
-  if (!t->codes || !t->absmax_q || !t->absmax_c2 || !t->absmax_mean) return QLORA_ERR_NULL;
-  if (!aligned16(t->codes) || !aligned16(t->absmax_q) || !aligned16(t->absmax_c2) ||
-      !aligned16(t->absmax_mean))
-    return QLORA_ERR_ALIGN;
+  if (t->blocksize2 != 0) {          // double quantization: E4M3 codes, c2, mean
+    if (!t->codes || !t->absmax_q || !t->absmax_c2 || !t->absmax_mean) return QLORA_ERR_NULL;
+    if (!aligned16(t->codes) || !aligned16(t->absmax_q) || !aligned16(t->absmax_c2) ||
+        !aligned16(t->absmax_mean))
+      return QLORA_ERR_ALIGN;
+  } else {                           // fp32 block constants
+    if (!t->codes || !t->absmax) return QLORA_ERR_NULL;
+    if (!aligned16(t->codes) || !aligned16(t->absmax)) return QLORA_ERR_ALIGN;
+  }
   return QLORA_OK;
+}
+
+size_t quantize_workspace_bytes(int64_t numel, bool double_quant) {
+  const int64_t nblocks = (numel + kBlock - 1) / kBlock;
+  const size_t partials = kMaxEncodeGrid * sizeof(double);
+  return double_quant ? round_up(static_cast<size_t>(nblocks) * 4, 256) + partials : partials;
+}
+
+EncodeTables encode_tables(const Nf4Tables& tabs) {
+  EncodeTables et;
+  for (int i = 0; i < kBuckets; ++i) {
+    et.bucket_thr[i] = i < kNumBuckets ? tabs.bucket_thr[i] : INFINITY;
+    et.bucket_base[i] = i < kNumBuckets ? tabs.bucket_base[i] : 15;
+    et.bucket_fast[i] = i < kNumBuckets ? tabs.bucket_fast[i] : (0x7F7FFFE0u | 16u);
+  }
+  et.fast = tabs.fast_ok ? 1 : 0;
+  return et;
 }
 
 qlora_status device_error_flag(uint32_t** flag) {
@@ -293,19 +404,27 @@ void qlora_get_codebook(float out[16]) {
   for (int i = 0; i < 16; ++i) out[i] = t.level[i];
 }
 
+qlora_status qlora_get_levels(int32_t quant_type, float out[16]) {
+  if (!out) return QLORA_ERR_NULL;
+  if (quant_type < 0 || quant_type >= kNumTypes) return QLORA_ERR_UNSUPPORTED;
+  const Nf4Tables& t = level_tables(quant_type);
+  for (int i = 0; i < 16; ++i) out[i] = t.level[i];
+  return QLORA_OK;
+}
+
 qlora_status qlora_nf4_sizes(int64_t rows, int64_t cols, int32_t blocksize, int32_t blocksize2,
                              size_t* codes_bytes, size_t* absmax_q_bytes, size_t* absmax_c2_bytes,
                              size_t* workspace_bytes) {
   if (rows < 0 || cols < 0 || rows > kMaxDim || cols > kMaxDim) return QLORA_ERR_SHAPE;
-  if (blocksize != kBlock || blocksize2 != kBlock2) return QLORA_ERR_UNSUPPORTED;
+  if (blocksize != kBlock || (blocksize2 != kBlock2 && blocksize2 != 0)) return QLORA_ERR_UNSUPPORTED;
+  const bool dq = blocksize2 != 0;
   const int64_t numel = rows * cols;
   const int64_t nblocks = (numel + kBlock - 1) / kBlock;
   const int64_t ngroups = (nblocks + kBlock2 - 1) / kBlock2;
   if (codes_bytes) *codes_bytes = static_cast<size_t>((numel + 1) / 2);
-  if (absmax_q_bytes) *absmax_q_bytes = static_cast<size_t>(nblocks);
-  if (absmax_c2_bytes) *absmax_c2_bytes = static_cast<size_t>(ngroups) * 4;
-  if (workspace_bytes)
-    *workspace_bytes = round_up(static_cast<size_t>(nblocks) * 4, 256) + kMaxEncodeGrid * sizeof(double);
+  if (absmax_q_bytes) *absmax_q_bytes = static_cast<size_t>(nblocks) * (dq ? 1 : 4);
+  if (absmax_c2_bytes) *absmax_c2_bytes = dq ? static_cast<size_t>(ngroups) * 4 : 0;
+  if (workspace_bytes) *workspace_bytes = quantize_workspace_bytes(numel, dq);
   return QLORA_OK;
 }
 
@@ -317,26 +436,20 @@ qlora_status qlora_quantize_nf4_dq(const uint16_t* W, const qlora_nf4_tensor* ou
   if (numel == 0) return QLORA_OK;
   if (!W || !workspace) return QLORA_ERR_NULL;
   if (!aligned16(W) || !aligned16(workspace)) return QLORA_ERR_ALIGN;
-  size_t need = 0;
-  qlora_nf4_sizes(out->rows, out->cols, kBlock, kBlock2, nullptr, nullptr, nullptr, &need);
-  if (workspace_bytes < need) return QLORA_ERR_WORKSPACE;
-  const Nf4Tables& tabs = nf4_tables();
+  const bool dq = out->blocksize2 != 0;
+  if (workspace_bytes < quantize_workspace_bytes(numel, dq)) return QLORA_ERR_WORKSPACE;
+  const Nf4Tables& tabs = level_tables(out->quant_type);
   if (!tabs.ok) return QLORA_ERR_UNSUPPORTED;
   DeviceInfo d;
   if ((st = device_info(&d)) != QLORA_OK) return st;
 
-  EncodeTables et;
-  for (int i = 0; i < kBuckets; ++i) {
-    et.bucket_thr[i] = i < kNumBuckets ? tabs.bucket_thr[i] : INFINITY;
-    et.bucket_base[i] = i < kNumBuckets ? tabs.bucket_base[i] : 15;
-    et.bucket_fast[i] = i < kNumBuckets ? tabs.bucket_fast[i] : (0x7F7FFFE0u | 16u);
-  }
-  et.fast = tabs.fast_ok ? 1 : 0;
-
+  const EncodeTables et = encode_tables(tabs);
   const int64_t nblocks = (numel + kBlock - 1) / kBlock;
-  float* c1buf = static_cast<float*>(workspace);
-  double* partials = reinterpret_cast<double*>(static_cast<uint8_t*>(workspace) +
-                                               round_up(static_cast<size_t>(nblocks) * 4, 256));
+  // with double quantization the block absmax values are scratch for
+  // k_double_quant; without it they are the stored constants themselves
+  float* c1buf = dq ? static_cast<float*>(workspace) : out->absmax;
+  double* partials = reinterpret_cast<double*>(
+      static_cast<uint8_t*>(workspace) + (dq ? round_up(static_cast<size_t>(nblocks) * 4, 256) : 0));
   const int64_t nvec = nblocks * 8;
   int grid = static_cast<int>((nvec + 255) / 256);
   const int wave = d.num_sms * encode_ctas_per_sm();           // one wave of resident CTAs
@@ -345,6 +458,7 @@ qlora_status qlora_quantize_nf4_dq(const uint16_t* W, const qlora_nf4_tensor* ou
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = counted(launch_encode(W, numel, et, out->codes, c1buf, partials, grid, s));
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  if (!dq) return QLORA_OK;
   const int64_t ngroups = (nblocks + kBlock2 - 1) / kBlock2;
   int grid2 = static_cast<int>((ngroups + 7) / 8);
   if (grid2 > d.num_sms * 4) grid2 = d.num_sms * 4;
@@ -368,7 +482,7 @@ qlora_status qlora_dequantize(const qlora_nf4_tensor* W, uint16_t* W_out, qlora_
   const int wave = d.num_sms * dequant_ctas_per_sm();          // one wave of resident CTAs
   if (grid > wave) grid = wave;
   return cuda_status(counted(launch_dequant(W->codes, W->absmax_q, W->absmax_c2, W->absmax_mean,
-                                            numel, codebook_param(), W_out, grid,
+                                            plain_absmax(W), numel, codebook_param(W->quant_type), W_out, grid,
                                             reinterpret_cast<cudaStream_t>(stream))));
 }
 
@@ -402,76 +516,46 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor* W, const uint16_t* X, int6
       (XA_out && !aligned16(XA_out)))
     return QLORA_ERR_ALIGN;
   if (!std::isfinite(s)) return QLORA_ERR_SHAPE;
-  const FwdLayout L = fwd_layout(sh);
-  if (workspace_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  // the size check uses the device-independent layout (an upper bound of the
+  // one the launch uses, which depends on the SM count)
+  if (workspace_bytes < fwd_layout(sh).total) return QLORA_ERR_WORKSPACE;
   DeviceInfo d;
   if ((st = device_info(&d)) != QLORA_OK) return st;
+  const FwdLayout L = fwd_layout(sh, d.num_sms);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
 
-  if (sh.decode) {
-    // Decode shapes: X A^T slices and the zeroed tile counters (k_xa_zero),
-    // then one pass over the packed weight that also writes Y (k_gemv, the
-    // programmatic dependent of k_xa_zero).
-    uint32_t* cnt = reinterpret_cast<uint32_t*>(ws + L.cnt);
-    const int m_tiles = static_cast<int>((sh.rows + gemv_tile_rows() - 1) / gemv_tile_rows());
-    float* xa_slices = reinterpret_cast<float*>(ws + L.xa_slices);
-    const int xa_splits = xa_splits_for(sh.r, sh.cols);
-    if (counted(launch_xa_zero(X, A, sh.m, sh.cols, sh.r, xa_slices, sh.rpad, xa_splits,
-                               reinterpret_cast<float*>(cnt), static_cast<int64_t>(m_tiles) * 8, cs)) !=
-        cudaSuccess)
-      return QLORA_ERR_CUDA;
-    CUtensorMap c_map, x_act;
-    if (!make_map_u8(&c_map, W->codes, sh.cols / 2, sh.rows, sh.cols / 2, 128, gemv_tile_rows(),
-                     CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&x_act, X, sh.cols, sh.m, sh.cols * 2, static_cast<uint32_t>(sh.m)))
-      return QLORA_ERR_CUDA;
-    GemvArgs ga{};
-    ga.qabs = W->absmax_q; ga.c2 = W->absmax_c2; ga.mean = W->absmax_mean;
-    ga.nw = sh.rows; ga.kw = sh.cols; ga.m = sh.m;
-    ga.slots = reinterpret_cast<float*>(ws + L.slots);
-    ga.cnt = cnt;
-    ga.xa_part = xa_slices; ga.ld_xa = sh.rpad; ga.r = sh.r; ga.lora_steps = sh.lora_steps;
-    ga.xa_splits = xa_splits;
-    ga.s = s; ga.lora_b = B; ga.y = Y; ga.xa_out = XA_out;
-    ga.m_tiles = m_tiles;
-    ga.steps = static_cast<int>((sh.cols / 64 + 3) / 4);
-    const CodebookParam cbp = codebook_param();
-    for (int i = 0; i < 16; ++i) ga.level[i] = cbp.level[i];
-    ga.err = d.err;
-    if (counted(launch_gemv(ga, c_map, x_act, d.num_sms, cs)) != cudaSuccess) return QLORA_ERR_CUDA;
-    return QLORA_OK;
-  }
+  if (sh.decode)
+    return run_decode_fwd(W, X, sh, A, B, nullptr, 1, s, Y, XA_out, ws, L, d, cs);
 
-  float* xa_acc = reinterpret_cast<float*>(ws + L.xa_acc);
+  // 1) X A^T (fp32 to XA_out when asked) and bf16(s X A^T), zero-padded to a
+  //    multiple of 64 columns, as the LoRA k-step operand of the fused GEMM
   uint16_t* sxa = reinterpret_cast<uint16_t*>(ws + L.sxa);
-  if (cudaMemsetAsync(ws, 0, L.fp32_end, cs) != cudaSuccess) return QLORA_ERR_CUDA;
-
-  // 1) XA = X A^T  (skinny tcgen05 GEMM, split-K into fp32)
+  const RankPlan xp = rank_plan(sh.m, sh.cols, sh.lora_steps, int((sh.m + 127) / 128) * sh.lora_steps, d.num_sms);
+  if (xp.splits > 1 && cudaMemsetAsync(ws, 0, L.clear_end, cs) != cudaSuccess) return QLORA_ERR_CUDA;
   CUtensorMap x_k, a_k;
   if (!make_map(&x_k, X, sh.cols, sh.m, sh.cols * 2, 128) ||
       !make_map(&a_k, A, sh.cols, sh.r, sh.cols * 2, 64))
     return QLORA_ERR_CUDA;
-  if ((st = run_skinny(false, false, x_k, a_k, sh.m, sh.r, sh.cols, xa_acc, sh.rpad, d, cs)) != QLORA_OK)
-    return st;
-  // 2) bf16(s XA), zero-padded to a multiple of 64 columns, as the LoRA k-step operand;
-  //    XA itself (fp32, unscaled) for the backward pass
-  if (counted(launch_convert_bf16(xa_acc, sh.m, sh.rpad, sh.rpad, sh.rpad, s, sxa, sh.rpad, d.num_sms, cs)) !=
-      cudaSuccess)
-    return QLORA_ERR_CUDA;
-  if (XA_out &&
-      counted(launch_convert_f32(xa_acc, sh.m, sh.r, sh.rpad, 1.0f, false, XA_out, sh.r, d.num_sms, cs)) !=
-          cudaSuccess)
-    return QLORA_ERR_CUDA;
+  RankArgs ra{};
+  ra.p[0] = rank_problem(xp, sh.m, sh.r, false, false, 0, reinterpret_cast<float*>(ws + L.rank_slots),
+                         reinterpret_cast<uint32_t*>(ws + L.rank_cnt));
+  ra.p[0].out_f32 = XA_out; ra.p[0].ld_f32 = sh.r;
+  ra.p[0].out_bf16 = sxa; ra.p[0].ld_bf16 = sh.rpad; ra.p[0].bf16_cols = sh.rpad; ra.p[0].bf16_scale = s;
+  ra.nprob = 1;
+  ra.total_units = xp.tiles() * xp.splits;
+  ra.err = d.err;
+  if (counted(launch_rank(ra, x_k, a_k, x_k, a_k, d.num_sms, cs)) != cudaSuccess) return QLORA_ERR_CUDA;
 
-  // 3) Y = X deq(W)^T + (s XA) B^T  (fused dequant GEMM)
-  const int bn = sh.decode ? 16 : 256;
+  // 2) Y = X deq(W)^T + (s XA) B^T  (fused dequant GEMM)
+  const int bn = 256;
   CUtensorMap x_act, sxa_map;
   if (!make_map(&x_act, X, sh.cols, sh.m, sh.cols * 2, bn) ||
       !make_map(&sxa_map, sxa, sh.rpad, sh.m, sh.rpad * 2, bn))
     return QLORA_ERR_CUDA;
   FusedArgs fa{};
   fa.codes = W->codes; fa.qabs = W->absmax_q; fa.c2 = W->absmax_c2; fa.mean = W->absmax_mean;
+  fa.absf = plain_absmax(W);
   fa.nw = sh.rows; fa.kw = sh.cols; fa.m = sh.m;
   fa.lora_w = B; fa.r = sh.r; fa.lora_steps = sh.lora_steps;
   fa.ldo = sh.rows; fa.mdim = sh.rows;
@@ -481,11 +565,35 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor* W, const uint16_t* X, int6
   fa.splits = 1;
   fa.m_group = m_group_for(fa.m_tiles, sh.cols);
   fa.out = Y; fa.out_acc = nullptr;
-  fa.cb = codebook_param();
+  fa.cb = codebook_param(W->quant_type);
   fa.err = d.err;
   if (fused_timed(FusedDir::kFwd, bn, fa, x_act, sxa_map, d.num_sms, cs) != cudaSuccess)
     return QLORA_ERR_CUDA;
   return QLORA_OK;
+}
+
+qlora_status qlora_linear_fwd_multi(const qlora_nf4_tensor* W, const uint16_t* X, int64_t M,
+                                    const uint16_t* A_stack, const uint16_t* B_stack, int32_t n_adapters,
+                                    const int32_t* adapter_idx, int32_t r, float s, uint16_t* Y,
+                                    float* XA_out, void* workspace, size_t workspace_bytes,
+                                    qlora_stream_t stream) {
+  LinearShape sh;
+  qlora_status st = check_linear(W, M, r, &sh);
+  if (st != QLORA_OK) return st;
+  if (!sh.decode || n_adapters < 1) return QLORA_ERR_SHAPE;
+  if (!X || !A_stack || !B_stack || !adapter_idx || !Y || !workspace) return QLORA_ERR_NULL;
+  if (!aligned16(X) || !aligned16(A_stack) || !aligned16(B_stack) || !aligned16(Y) || !aligned16(workspace) ||
+      (XA_out && !aligned16(XA_out)) || (reinterpret_cast<uintptr_t>(adapter_idx) & 3u) != 0)
+    return QLORA_ERR_ALIGN;
+  if (!std::isfinite(s)) return QLORA_ERR_SHAPE;
+  // the size check uses the device-independent layout (an upper bound of the
+  // one the launch uses, which depends on the SM count)
+  if (workspace_bytes < fwd_layout(sh).total) return QLORA_ERR_WORKSPACE;
+  DeviceInfo d;
+  if ((st = device_info(&d)) != QLORA_OK) return st;
+  const FwdLayout L = fwd_layout(sh, d.num_sms);
+  return run_decode_fwd(W, X, sh, A_stack, B_stack, adapter_idx, n_adapters, s, Y, XA_out,
+                        static_cast<uint8_t*>(workspace), L, d, reinterpret_cast<cudaStream_t>(stream));
 }
 
 qlora_status qlora_linear_bwd(const qlora_nf4_tensor* W, const uint16_t* X, const uint16_t* dY,
@@ -500,49 +608,56 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor* W, const uint16_t* X, cons
       !aligned16(dB) || !aligned16(workspace) || (XA && !aligned16(XA)) || (dX && !aligned16(dX)))
     return QLORA_ERR_ALIGN;
   if (!std::isfinite(s)) return QLORA_ERR_SHAPE;
-  const BwdLayout L = bwd_layout(sh);
-  if (workspace_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  if (workspace_bytes < bwd_layout(sh).total) return QLORA_ERR_WORKSPACE;
   DeviceInfo d;
   if ((st = device_info(&d)) != QLORA_OK) return st;
+  const BwdLayout L = bwd_layout(sh, d.num_sms);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* g_acc = reinterpret_cast<float*>(ws + L.g_acc);
-  float* xa_acc = reinterpret_cast<float*>(ws + L.xa_acc);
   float* dx_acc = reinterpret_cast<float*>(ws + L.dx_acc);
-  float* da_acc = reinterpret_cast<float*>(ws + L.da_acc);
-  float* db_acc = reinterpret_cast<float*>(ws + L.db_acc);
+  float* g32 = sh.decode ? reinterpret_cast<float*>(ws + L.g) : nullptr;     // fp32 G and X A^T: few-token grads
+  float* xa32 = sh.decode ? reinterpret_cast<float*>(ws + L.xa) : nullptr;
   uint16_t* sg = reinterpret_cast<uint16_t*>(ws + L.sg);
-  uint16_t* sxa = reinterpret_cast<uint16_t*>(ws + L.xa);
+  uint16_t* sxa = reinterpret_cast<uint16_t*>(ws + L.sxa);
+  const bool recompute = XA == nullptr;
 
-  if (cudaMemsetAsync(ws, 0, L.fp32_end, cs) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (L.clear_end && cudaMemsetAsync(ws, 0, L.clear_end, cs) != cudaSuccess) return QLORA_ERR_CUDA;
 
-  // 1) G = dY B   (contraction over rows; B [rows, r] is the MN-major operand)
-  CUtensorMap dy_k, b_mn;
+  // 1) G = dY B -> bf16(s G) (+ fp32 G for few tokens), and X A^T -> bf16(s X A^T)
+  //    (recomputed when not supplied, else converted from the caller's fp32)
+  CUtensorMap dy_k, b_mn, x_k, a_k;
   if (!make_map(&dy_k, dY, sh.rows, sh.m, sh.rows * 2, 128) ||
-      !make_map(&b_mn, B, sh.r, sh.rows, sh.r * 2, 64))
+      !make_map(&b_mn, B, sh.r, sh.rows, sh.r * 2, 64) ||
+      !make_map(&x_k, X, sh.cols, sh.m, sh.cols * 2, 128) ||
+      !make_map(&a_k, A, sh.cols, sh.r, sh.cols * 2, 64))
     return QLORA_ERR_CUDA;
-  if ((st = run_skinny(false, true, dy_k, b_mn, sh.m, sh.r, sh.rows, g_acc, sh.rpad, d, cs)) != QLORA_OK)
-    return st;
-  if (counted(launch_convert_bf16(g_acc, sh.m, sh.rpad, sh.rpad, sh.rpad, s, sg, sh.rpad, d.num_sms, cs)) !=
-      cudaSuccess)
-    return QLORA_ERR_CUDA;
-
-  // 2) XA in fp32: as supplied by the forward, or recomputed
-  const float* xa = XA;
-  int64_t ld_xa = sh.r;
-  if (!xa) {
-    CUtensorMap x_k, a_k;
-    if (!make_map(&x_k, X, sh.cols, sh.m, sh.cols * 2, 128) ||
-        !make_map(&a_k, A, sh.cols, sh.r, sh.cols * 2, 64))
-      return QLORA_ERR_CUDA;
-    if ((st = run_skinny(false, false, x_k, a_k, sh.m, sh.r, sh.cols, xa_acc, sh.rpad, d, cs)) !=
-        QLORA_OK)
-      return st;
-    xa = xa_acc;
-    ld_xa = sh.rpad;
+  {
+    RankArgs ra{};
+    uint32_t* cnt = reinterpret_cast<uint32_t*>(ws + L.cnt1);
+    float* slots = reinterpret_cast<float*>(ws + L.slots1);
+    ra.p[0] = rank_problem(L.g_plan, sh.m, sh.r, false, true, 0, slots, cnt);
+    ra.p[0].out_f32 = g32; ra.p[0].ld_f32 = sh.rpad;
+    ra.p[0].out_bf16 = sg; ra.p[0].ld_bf16 = sh.rpad; ra.p[0].bf16_cols = sh.rpad; ra.p[0].bf16_scale = s;
+    ra.nprob = 1;
+    ra.total_units = L.g_plan.tiles() * L.g_plan.splits;
+    if (recompute) {
+      ra.p[1] = rank_problem(L.xa_plan, sh.m, sh.r, false, false, ra.total_units,
+                             slots + rank_slot_bytes(L.g_plan.tiles(), L.g_plan.splits) / 4,
+                             cnt + L.g_plan.tiles());
+      ra.p[1].out_f32 = xa32; ra.p[1].ld_f32 = sh.rpad;
+      ra.p[1].out_bf16 = sh.decode ? nullptr : sxa;
+      ra.p[1].ld_bf16 = sh.rpad; ra.p[1].bf16_cols = sh.rpad; ra.p[1].bf16_scale = s;
+      ra.nprob = 2;
+      ra.total_units += L.xa_plan.tiles() * L.xa_plan.splits;
+    } else if (!sh.decode) {
+      ra.cvt_in = XA; ra.cvt_rows = sh.m; ra.cvt_cols = sh.r; ra.cvt_ld_in = sh.r;
+      ra.cvt_out = sxa; ra.cvt_ld_out = sh.rpad; ra.cvt_cols_out = sh.rpad; ra.cvt_scale = s;
+    }
+    ra.err = d.err;
+    if (counted(launch_rank(ra, dy_k, b_mn, x_k, a_k, d.num_sms, cs)) != cudaSuccess) return QLORA_ERR_CUDA;
   }
 
-  // 3) dX = dY deq(W) + (s G) A   (fused dequant GEMM, deq(W)^T as the MN-major operand)
+  // 2) dX = dY deq(W) + (s G) A   (fused dequant GEMM, deq(W)^T as the MN-major operand)
   if (dX) {
     const int bn = sh.decode ? 16 : 256;
     CUtensorMap dy_act, sg_map;
@@ -551,6 +666,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor* W, const uint16_t* X, cons
       return QLORA_ERR_CUDA;
     FusedArgs fa{};
     fa.codes = W->codes; fa.qabs = W->absmax_q; fa.c2 = W->absmax_c2; fa.mean = W->absmax_mean;
+    fa.absf = plain_absmax(W);
     fa.nw = sh.rows; fa.kw = sh.cols; fa.m = sh.m;
     fa.lora_w = A; fa.r = sh.r; fa.lora_steps = sh.lora_steps;
     fa.ldo = sh.cols; fa.mdim = sh.cols;
@@ -560,7 +676,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor* W, const uint16_t* X, cons
     fa.splits = sh.decode ? choose_splits(fa.m_tiles, fa.ksteps, d.num_sms) : 1;
     fa.m_group = m_group_for(fa.m_tiles, sh.rows);
     fa.out = dX; fa.out_acc = dx_acc;
-    fa.cb = codebook_param();
+    fa.cb = codebook_param(W->quant_type);
     fa.err = d.err;
     if (fused_timed(FusedDir::kBwd, bn, fa, dy_act, sg_map, d.num_sms, cs) != cudaSuccess)
       return QLORA_ERR_CUDA;
@@ -570,34 +686,37 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor* W, const uint16_t* X, cons
       return QLORA_ERR_CUDA;
   }
 
-  // 4) LoRA gradients.  Few tokens: fp32 on CUDA cores from the fp32 G and XA.
+  // 3) LoRA gradients.  Few tokens: fp32 on CUDA cores from the fp32 G and X A^T.
   if (sh.decode) {
-    if (counted(launch_small_grads(g_acc, sh.rpad, xa, ld_xa, X, dY, sh.m, sh.rows, sh.cols, sh.r, s,
+    const float* xa = recompute ? xa32 : XA;
+    const int64_t ld_xa = recompute ? sh.rpad : sh.r;
+    if (counted(launch_small_grads(g32, sh.rpad, xa, ld_xa, X, dY, sh.m, sh.rows, sh.cols, sh.r, s,
                                    dA, dB, d.num_sms, cs)) != cudaSuccess)
       return QLORA_ERR_CUDA;
     return QLORA_OK;
   }
-  //    Many tokens: tcgen05 contractions over the tokens with bf16 operands.
-  //    dB = dY^T (s XA)  ([rows, r]; both operands MN-major)
-  if (counted(launch_convert_bf16(xa, sh.m, sh.r, ld_xa, sh.rpad, s, sxa, sh.rpad, d.num_sms, cs)) != cudaSuccess)
-    return QLORA_ERR_CUDA;
-  CUtensorMap dy_mn, sxa_mn;
+  //    Many tokens, one launch of two contractions over the tokens (bf16 operands):
+  //    dB = dY^T (s X A^T) [rows, r] and dA = (X^T (s G))^T [r, cols], stored transposed.
+  CUtensorMap dy_mn, sxa_mn, x_mn, sg_mn;
   if (!make_map(&dy_mn, dY, sh.rows, sh.m, sh.rows * 2, 64) ||
-      !make_map(&sxa_mn, sxa, sh.rpad, sh.m, sh.rpad * 2, 64))
-    return QLORA_ERR_CUDA;
-  if ((st = run_skinny(true, true, dy_mn, sxa_mn, sh.rows, sh.r, sh.m, db_acc, sh.rpad, d, cs)) != QLORA_OK)
-    return st;
-  //    dA^T = X^T (s G)  ([cols, r])
-  CUtensorMap x_mn, sg_mn;
-  if (!make_map(&x_mn, X, sh.cols, sh.m, sh.cols * 2, 64) ||
+      !make_map(&sxa_mn, sxa, sh.rpad, sh.m, sh.rpad * 2, 64) ||
+      !make_map(&x_mn, X, sh.cols, sh.m, sh.cols * 2, 64) ||
       !make_map(&sg_mn, sg, sh.rpad, sh.m, sh.rpad * 2, 64))
     return QLORA_ERR_CUDA;
-  if ((st = run_skinny(true, true, x_mn, sg_mn, sh.cols, sh.r, sh.m, da_acc, sh.rpad, d, cs)) != QLORA_OK)
-    return st;
-  if (counted(launch_convert_f32(db_acc, sh.rows, sh.r, sh.rpad, 1.0f, false, dB, sh.r, d.num_sms, cs)) != cudaSuccess)
-    return QLORA_ERR_CUDA;
-  if (counted(launch_convert_f32(da_acc, sh.cols, sh.r, sh.rpad, 1.0f, true, dA, sh.cols, d.num_sms, cs)) != cudaSuccess)
-    return QLORA_ERR_CUDA;
+  RankArgs rb{};
+  uint32_t* cnt2 = reinterpret_cast<uint32_t*>(ws + L.cnt2);
+  float* slots2 = reinterpret_cast<float*>(ws + L.slots2);
+  rb.p[0] = rank_problem(L.db_plan, sh.rows, sh.r, true, true, 0, slots2, cnt2);
+  rb.p[0].out_f32 = dB; rb.p[0].ld_f32 = sh.r;
+  const int u0 = L.db_plan.tiles() * L.db_plan.splits;
+  rb.p[1] = rank_problem(L.da_plan, sh.cols, sh.r, true, true, u0,
+                         slots2 + rank_slot_bytes(L.db_plan.tiles(), L.db_plan.splits) / 4,
+                         cnt2 + L.db_plan.tiles());
+  rb.p[1].out_f32 = dA; rb.p[1].ld_f32 = sh.cols; rb.p[1].transpose = 1;
+  rb.nprob = 2;
+  rb.total_units = u0 + L.da_plan.tiles() * L.da_plan.splits;
+  rb.err = d.err;
+  if (counted(launch_rank(rb, dy_mn, sxa_mn, x_mn, sg_mn, d.num_sms, cs)) != cudaSuccess) return QLORA_ERR_CUDA;
   return QLORA_OK;
 }
 

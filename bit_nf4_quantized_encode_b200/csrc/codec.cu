@@ -11,6 +11,9 @@
 //   per tensor      mu = float(double-sum(c1) / nblocks);
 //   per 256 c1      c2 = max |c1 - mu|;  q = E4M3_RNE(float((c1-mu)/c2) * 448), 0 if c2 == 0.
 //   dequant         c1' = fma(e4m3(q), c2/448, mu);  w' = bf16_RNE(L[code] * c1').
+//   Without double quantization the fp32 c1 is stored and used as the
+//   constant (w' = bf16_RNE(L[code] * c1)); the levels L are those of the
+//   weight's 4-bit type (NF4, or the FP4 / INT4 tables it is compared with).
 // Every float operation uses an explicitly rounded intrinsic so the compiler
 // cannot contract or reorder it: the results are bit-identical to any
 // implementation that performs the same IEEE operations.
@@ -258,9 +261,11 @@ __global__ void __launch_bounds__(256) k_double_quant(const float* __restrict__ 
 // SM that keeps about 64 KB of codes in flight per SM, above HBM's
 // bandwidth-delay product.  A ragged last chunk is expanded element by element.
 constexpr int kDqUnroll = 8;
-__device__ __forceinline__ void dequant_chunk(const uint4 cw, uint32_t q, float c2v, float mu,
+// c2v is the group's c2 with double quantization, the block's own fp32
+// constant without it (plain).
+__device__ __forceinline__ void dequant_chunk(const uint4 cw, uint32_t q, float c2v, float mu, bool plain,
                                               const CodebookParam& cb, uint4 (&o)[4]) {
-  const float c1p = block_constant(q, __fdiv_rn(c2v, 448.0f), mu);
+  const float c1p = plain ? c2v : block_constant(q, __fdiv_rn(c2v, 448.0f), mu);
   const ByteTables t = make_tables(cb.level, c1p);
   o[0] = expand8(cw.x, t);
   o[1] = expand8(cw.y, t);
@@ -275,10 +280,11 @@ __device__ __forceinline__ void dequant_chunk(const uint4 cw, uint32_t q, float 
 __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ codes,
                                                  const uint8_t* __restrict__ qabs,
                                                  const float* __restrict__ c2, const float* __restrict__ mean,
-                                                 int64_t numel, CodebookParam cb,
-                                                 uint16_t* __restrict__ out) {
+                                                 const float* __restrict__ absf, int64_t numel,
+                                                 CodebookParam cb, uint16_t* __restrict__ out) {
   __shared__ __align__(16) uint8_t s_out[8][32 * 80];
-  const float mu = __ldg(mean);
+  const bool plain = absf != nullptr;                // fp32 block constants, no double quantization
+  const float mu = plain ? 0.0f : __ldg(mean);
   const int64_t nfull = numel / 32;                  // chunks of 32 real weights
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const uint4* cw4 = reinterpret_cast<const uint4*>(codes);
@@ -299,8 +305,12 @@ __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ cod
       c2v[u] = 0.0f;
       if (c < nfull) {
         cw[u] = __ldg(cw4 + c);
-        qv[u] = __ldg(qabs + (c >> 1));
-        c2v[u] = __ldg(c2 + (c >> 9));
+        if (plain) {
+          c2v[u] = __ldg(absf + (c >> 1));
+        } else {
+          qv[u] = __ldg(qabs + (c >> 1));
+          c2v[u] = __ldg(c2 + (c >> 9));
+        }
       }
     }
 #pragma unroll
@@ -308,7 +318,7 @@ __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ cod
       const int64_t c = ch + u * stride;
       const int64_t wc0 = c - lane;                  // the warp's first chunk
       uint4 o[4];
-      dequant_chunk(cw[u], qv[u], c2v[u], mu, cb, o);
+      dequant_chunk(cw[u], qv[u], c2v[u], mu, plain, cb, o);
 #pragma unroll
       for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4*>(st + lane * 80 + k * 16) = o[k];
       __syncwarp();
@@ -324,7 +334,7 @@ __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ cod
   // ragged last chunk
   if (blockIdx.x == 0 && threadIdx.x == 0 && nfull * 32 < numel) {
     const int64_t blk = nfull >> 1;
-    const float c1p = block_constant(qabs[blk], __fdiv_rn(c2[blk >> 8], 448.0f), mu);
+    const float c1p = plain ? absf[blk] : block_constant(qabs[blk], __fdiv_rn(c2[blk >> 8], 448.0f), mu);
     for (int64_t e = nfull * 32; e < numel; ++e) {
       const uint32_t byte = codes[e >> 1];
       const uint32_t code = (e & 1) ? (byte & 15u) : (byte >> 4);
@@ -370,9 +380,9 @@ int encode_ctas_per_sm() {
 }
 
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* qabs, const float* c2,
-                           const float* mean, int64_t numel, const CodebookParam& cb, uint16_t* out,
-                           int grid, cudaStream_t stream) {
-  k_dequant<<<grid, 256, 0, stream>>>(codes, qabs, c2, mean, numel, cb, out);
+                           const float* mean, const float* absf, int64_t numel, const CodebookParam& cb,
+                           uint16_t* out, int grid, cudaStream_t stream) {
+  k_dequant<<<grid, 256, 0, stream>>>(codes, qabs, c2, mean, absf, numel, cb, out);
   return cudaGetLastError();
 }
 

@@ -16,7 +16,7 @@ struct EncodeTables {
   int fast;                         // nonzero: the reciprocal path may be used
 };
 
-// The 16 NF4 levels, passed by value.
+// The 16 levels of the weight's 4-bit type, passed by value.
 struct CodebookParam {
   float level[16];
 };
@@ -31,8 +31,10 @@ int dequant_ctas_per_sm();
 cudaError_t launch_double_quant(const float* c1buf, int64_t nblocks, const double* partials,
                                 int npartials, uint8_t* q, float* c2, float* mean, int grid,
                                 cudaStream_t stream);
+// absf: the fp32 block constants of a weight stored without double
+// quantization (qabs, c2 and mean are then unused), else NULL.
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* qabs, const float* c2,
-                           const float* mean, int64_t numel, const CodebookParam& cb, uint16_t* out,
-                           int grid, cudaStream_t stream);
+                           const float* mean, const float* absf, int64_t numel, const CodebookParam& cb,
+                           uint16_t* out, int grid, cudaStream_t stream);
 
 }  // namespace qlora

@@ -93,7 +93,7 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void* p, uint64_t pol) {
 struct DqLoad {
   uint4 c0, c1;        // 64 packed codes (32 bytes)
   uint32_t q;          // E4M3 block constant
-  float c2;            // second-level absmax of its group
+  float c2;            // second-level absmax of its group (without double quantization: c1 itself)
   bool valid;
 };
 
@@ -115,8 +115,13 @@ __device__ __forceinline__ DqLoad dq_load(const FusedArgs& a, int m0, int kstep,
     d.c0 = ldg_nc_v4(p, pol);
     d.c1 = ldg_nc_v4(p + 16, pol);
     const int64_t blk = e >> 6;
-    d.q = __ldg(a.qabs + blk);
-    d.c2 = __ldg(a.c2 + (blk >> 8));
+    if (a.absf) {                 // no double quantization: the constant itself
+      d.q = 0;
+      d.c2 = __ldg(a.absf + blk);
+    } else {
+      d.q = __ldg(a.qabs + blk);
+      d.c2 = __ldg(a.c2 + (blk >> 8));
+    }
   }
   return d;
 }
@@ -130,7 +135,7 @@ __device__ __forceinline__ uint32_t task_row_base(int t, uint32_t& swz_row) {
 }
 
 template <int kDir>
-__device__ __forceinline__ void dq_store(uint32_t sA, int t, const DqLoad& d, float mu,
+__device__ __forceinline__ void dq_store(uint32_t sA, int t, const DqLoad& d, float mu, bool plain,
                                          const CodebookParam& cb) {
   uint32_t r;
   const uint32_t base = sA + task_row_base<kDir>(t, r);
@@ -140,7 +145,7 @@ __device__ __forceinline__ void dq_store(uint32_t sA, int t, const DqLoad& d, fl
     for (int c = 0; c < 8; ++c) st_shared_v4(base + (((c ^ (r & 7)) << 4)), z);
     return;
   }
-  const float c1p = block_constant(d.q, __fdiv_rn(d.c2, 448.0f), mu);
+  const float c1p = plain ? d.c2 : block_constant(d.q, __fdiv_rn(d.c2, 448.0f), mu);
   const ByteTables tb = make_tables(cb.level, c1p);
   const uint32_t w[8] = {d.c0.x, d.c0.y, d.c0.z, d.c0.w, d.c1.x, d.c1.y, d.c1.z, d.c1.w};
 #pragma unroll
@@ -232,7 +237,8 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
     // ------------------------------------------------ dequant producers
     const int group = warp >> 2;              // warps 4g .. 4g+3
     const int t = threadIdx.x & 127;
-    const float mu = __ldg(a.mean);
+    const bool plain = a.absf != nullptr;
+    const float mu = plain ? 0.0f : __ldg(a.mean);
     const uint64_t codes_pol = l2_evict_last_policy();
     uint32_t gctr = 0;
     bool alive = true;
@@ -249,7 +255,7 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
         if (j + kDequantGroups < w.kmain) next = dq_load<kDir>(a, m0, w.kbeg + j + kDequantGroups, t, codes_pol);
         if (!mbar_wait(&empty[stage], phase ^ 1u, a.err)) { alive = false; break; }
         const uint32_t sA = smem0 + stage * kStageBytes;
-        if (j < w.kmain) dq_store<kDir>(sA, t, cur, mu, a.cb);
+        if (j < w.kmain) dq_store<kDir>(sA, t, cur, mu, plain, a.cb);
         else lora_store<kDir>(a, sA, m0, j - w.kmain, t);
         fence_proxy_async_smem();
         mbar_arrive(&full_a[stage]);
@@ -363,165 +369,11 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
   }
 }
 
-// ------------------------------------------------------------------ skinny GEMM
-constexpr int kSkStages = 6;
-constexpr int kSkABytes = 128 * 128;     // 128 x 64 bf16
-constexpr int kSkBBytes = 64 * 128;      // 64 x 64 bf16
-constexpr int kSkStageBytes = kSkABytes + kSkBBytes;
-constexpr int kSkThreads = 6 * 32;       // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
-constexpr uint32_t kSkTmemCols = 128;    // two 64-column accumulators
-constexpr size_t kSkSmem = 1024 + kSkStages * kSkStageBytes + 256;
-
-template <bool kAMN, bool kBMN>
-__global__ void __launch_bounds__(kSkThreads, 1)
-k_skinny(const SkinnyArgs a, const __grid_constant__ CUtensorMap amap,
-         const __grid_constant__ CUtensorMap bmap) {
-  constexpr uint32_t kIdesc = idesc_bf16(128, 64, kAMN, kBMN);
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t smem0 = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  uint8_t* smem_gen = smem_raw + (smem0 - smem_u32(smem_raw));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_gen + kSkStages * kSkStageBytes);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + kSkStages;
-  uint64_t* acc_full = bars + 2 * kSkStages;
-  uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int nunits = a.m_tiles * a.n_tiles * a.splits;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kSkStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 128);
-    }
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, kSkTmemCols);
-    tmem_relinquish();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&amap);
-    tma_prefetch_desc(&bmap);
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-
-  auto unit_range = [&](int u, int& mt, int& nt, int& kbeg, int& nk) {
-    const int sp = u % a.splits;
-    const int rest = u / a.splits;
-    nt = rest % a.n_tiles;
-    mt = rest / a.n_tiles;
-    kbeg = static_cast<int>((static_cast<int64_t>(a.ksteps) * sp) / a.splits);
-    nk = static_cast<int>((static_cast<int64_t>(a.ksteps) * (sp + 1)) / a.splits) - kbeg;
-  };
-
-  if (warp == 0) {
-    if (lane == 0) {
-      uint32_t it = 0;
-      bool alive = true;
-      for (int u = blockIdx.x; u < nunits && alive; u += gridDim.x) {
-        int mt, nt, kbeg, nk;
-        unit_range(u, mt, nt, kbeg, nk);
-        for (int j = 0; j < nk; ++j, ++it) {
-          const uint32_t stage = it % kSkStages, phase = (it / kSkStages) & 1u;
-          if (!mbar_wait(&empty[stage], phase ^ 1u, a.err)) { alive = false; break; }
-          uint8_t* sA = smem_gen + stage * kSkStageBytes;
-          uint8_t* sB = sA + kSkABytes;
-          const int k0 = (kbeg + j) * 64;
-          mbar_arrive_expect_tx(&full[stage], kSkStageBytes);
-          if (kAMN) {   // A^T stored [k][m]: two 64-wide MN boxes
-            tma_load_2d(sA, &amap, mt * 128, k0, &full[stage]);
-            tma_load_2d(sA + 8192, &amap, mt * 128 + 64, k0, &full[stage]);
-          } else {
-            tma_load_2d(sA, &amap, k0, mt * 128, &full[stage]);
-          }
-          if (kBMN) tma_load_2d(sB, &bmap, nt * 64, k0, &full[stage]);
-          else tma_load_2d(sB, &bmap, k0, nt * 64, &full[stage]);
-        }
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      uint32_t it = 0, uctr = 0;
-      bool alive = true;
-      for (int u = blockIdx.x; u < nunits && alive; u += gridDim.x, ++uctr) {
-        int mt, nt, kbeg, nk;
-        unit_range(u, mt, nt, kbeg, nk);
-        const uint32_t ab = uctr & 1u, aphase = (uctr >> 1) & 1u;
-        if (!mbar_wait(&acc_empty[ab], aphase ^ 1u, a.err)) break;
-        tc_fence_after();
-        for (int j = 0; j < nk; ++j, ++it) {
-          const uint32_t stage = it % kSkStages, phase = (it / kSkStages) & 1u;
-          if (!mbar_wait(&full[stage], phase, a.err)) { alive = false; break; }
-          tc_fence_after();
-          const uint32_t sA = smem0 + stage * kSkStageBytes;
-          const uint32_t sB = sA + kSkABytes;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t adesc = kAMN ? smem_desc_sw128(sA + kk * 2048, 8192, 1024)
-                                        : smem_desc_sw128(sA + kk * 32, 16, 1024);
-            const uint64_t bdesc = kBMN ? smem_desc_sw128(sB + kk * 2048, 8192, 1024)
-                                        : smem_desc_sw128(sB + kk * 32, 16, 1024);
-            mma_bf16_ss(tmem_base + ab * 64, adesc, bdesc, kIdesc, (j | kk) != 0 ? 1u : 0u);
-          }
-          mma_commit(&empty[stage]);
-        }
-        if (alive) mma_commit(&acc_full[ab]);
-      }
-    }
-  } else {
-    const int quarter = warp & 3;            // warps 2,3,4,5 -> quarters 2,3,0,1
-    uint32_t uctr = 0;
-    for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++uctr) {
-      int mt, nt, kbeg, nk;
-      unit_range(u, mt, nt, kbeg, nk);
-      const uint32_t ab = uctr & 1u, aphase = (uctr >> 1) & 1u;
-      if (!mbar_wait(&acc_full[ab], aphase, a.err)) break;
-      tc_fence_after();
-      const int64_t row = static_cast<int64_t>(mt) * 128 + quarter * 32 + lane;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + ab * 64;
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(taddr + cc * 32, v);
-        tmem_wait_ld();
-        if (row < a.mdim) {
-          float* dst = a.acc + row * a.ld_acc;
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int64_t col = static_cast<int64_t>(nt) * 64 + cc * 32 + c;
-            if (col < a.ndim) atomicAdd(dst + col, __uint_as_float(v[c]));
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[ab]);
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, kSkTmemCols);
-  }
-}
-
 // ------------------------------------------------------------------ converts
 __device__ __forceinline__ void store_out(uint16_t* p, float v) {
   const __nv_bfloat16 b = __float2bfloat16_rn(v);
   *p = *reinterpret_cast<const uint16_t*>(&b);
 }
-__device__ __forceinline__ void store_out(float* p, float v) { *p = v; }
 
 template <typename T>
 __global__ void k_convert(const float* __restrict__ in, int64_t rows, int64_t cols_in, int64_t ld_in,
@@ -532,17 +384,6 @@ __global__ void k_convert(const float* __restrict__ in, int64_t rows, int64_t co
     const int64_t i = o / cols_out, j = o % cols_out;
     const float v = j < cols_in ? __fmul_rn(in[i * ld_in + j], scale) : 0.0f;
     store_out(out + i * ld_out + j, v);
-  }
-}
-
-__global__ void k_convert_t(const float* __restrict__ in, int64_t rows, int64_t cols, int64_t ld_in,
-                            float scale, float* __restrict__ out, int64_t ld_out) {
-  // consecutive threads walk i, the contiguous index of the output
-  const int64_t n = rows * cols;
-  for (int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; o < n;
-       o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t j = o / rows, i = o % rows;
-    out[j * ld_out + i] = __fmul_rn(in[i * ld_in + j], scale);
   }
 }
 
@@ -608,18 +449,6 @@ cudaError_t launch_fused_t(const FusedArgs& args, const CUtensorMap& act, const 
   return cudaGetLastError();
 }
 
-template <bool kAMN, bool kBMN>
-cudaError_t launch_skinny_t(const SkinnyArgs& args, const CUtensorMap& am, const CUtensorMap& bm,
-                            int num_sms, cudaStream_t stream) {
-  static std::atomic<uint64_t> attr_done{0};
-  cudaError_t e = ensure_smem_attr(k_skinny<kAMN, kBMN>, kSkSmem, attr_done);
-  if (e != cudaSuccess) return e;
-  const int nunits = args.m_tiles * args.n_tiles * args.splits;
-  const int grid = nunits < num_sms ? nunits : num_sms;
-  k_skinny<kAMN, kBMN><<<grid, kSkThreads, kSkSmem, stream>>>(args, am, bm);
-  return cudaGetLastError();
-}
-
 }  // namespace
 
 cudaError_t launch_fused(FusedDir dir, int token_tile, const FusedArgs& args, const CUtensorMap& act,
@@ -634,14 +463,6 @@ cudaError_t launch_fused(FusedDir dir, int token_tile, const FusedArgs& args, co
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_skinny(bool a_mn, bool b_mn, const SkinnyArgs& args, const CUtensorMap& am,
-                          const CUtensorMap& bm, int num_sms, cudaStream_t stream) {
-  if (!a_mn && !b_mn) return launch_skinny_t<false, false>(args, am, bm, num_sms, stream);
-  if (!a_mn && b_mn) return launch_skinny_t<false, true>(args, am, bm, num_sms, stream);
-  if (a_mn && b_mn) return launch_skinny_t<true, true>(args, am, bm, num_sms, stream);
-  return launch_skinny_t<true, false>(args, am, bm, num_sms, stream);
-}
-
 cudaError_t launch_convert_bf16(const float* in, int64_t rows, int64_t cols_in, int64_t ld_in,
                                 int64_t cols_out, float scale, uint16_t* out, int64_t ld_out, int num_sms,
                                 cudaStream_t stream) {
@@ -649,17 +470,6 @@ cudaError_t launch_convert_bf16(const float* in, int64_t rows, int64_t cols_in, 
   if (n == 0) return cudaSuccess;
   k_convert<uint16_t><<<grid_for(n, num_sms), 256, 0, stream>>>(in, rows, cols_in, ld_in, cols_out, scale,
                                                              out, ld_out);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_convert_f32(const float* in, int64_t rows, int64_t cols, int64_t ld_in, float scale,
-                               bool transpose, float* out, int64_t ld_out, int num_sms, cudaStream_t stream) {
-  const int64_t n = rows * cols;
-  if (n == 0) return cudaSuccess;
-  if (transpose)
-    k_convert_t<<<grid_for(n, num_sms), 256, 0, stream>>>(in, rows, cols, ld_in, scale, out, ld_out);
-  else
-    k_convert<float><<<grid_for(n, num_sms), 256, 0, stream>>>(in, rows, cols, ld_in, cols, scale, out, ld_out);
   return cudaGetLastError();
 }
 

@@ -8,9 +8,8 @@
 //    (MN-major).  The rank-r LoRA up-projection is appended as extra k-steps
 //    whose A operand is the LoRA weight and whose B operand is the (scaled)
 //    rank-r activation.
-//  * skinny GEMM: D[mdim x 64] = A x B^T over a long contraction, both operands
-//    by TMA (K- or MN-major), split-K with fp32 atomic accumulation; used for
-//    the rank-r LoRA contractions X A^T, dY B, dY^T (XA), G^T X.
+//  The rank-r LoRA contractions (X A^T, dY B, dY^T (s X A^T), X^T (s dY B))
+//  are in lora.cu.
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -28,6 +27,7 @@ struct FusedArgs {
   const uint8_t* qabs;       // E4M3 block constants
   const float* c2;           // per-group second-level absmax
   const float* mean;         // per-tensor mean of the block constants
+  const float* absf;         // fp32 block constants (no double quantization), else null
   int64_t nw, kw;            // W shape (out, in)
   int64_t m;                 // token rows
   const uint16_t* lora_w;    // fwd: LoRA B [nw, r]; bwd: LoRA A [r, kw] (bf16)
@@ -44,32 +44,16 @@ struct FusedArgs {
   uint32_t* err;             // device error flag
 };
 
-struct SkinnyArgs {
-  int64_t mdim, ndim;        // D extent (ndim <= 64 per n-tile)
-  int ksteps;                // contraction / 64 (rounded up)
-  int m_tiles, n_tiles, splits;
-  float* acc;                // fp32 [mdim, ld_acc], accumulated with atomics
-  int64_t ld_acc;
-  uint32_t* err;
-};
-
 // Token tile of the fused kernel: 256 for prefill-shaped calls, 16 for
 // decode-shaped calls (M <= 16).
 cudaError_t launch_fused(FusedDir dir, int token_tile, const FusedArgs& args, const CUtensorMap& act,
                          const CUtensorMap& lora_act, int num_sms, cudaStream_t stream);
-cudaError_t launch_skinny(bool a_mn_major, bool b_mn_major, const SkinnyArgs& args,
-                          const CUtensorMap& a_map, const CUtensorMap& b_map, int num_sms,
-                          cudaStream_t stream);
-
-// out[i * ld_out + j] = T(scale * in[i * ld_in + j]) for j < cols_in, 0 for
-// cols_in <= j < cols_out (i < rows); T is bf16 or fp32.  With `transpose`
-// the element goes to out[j * ld_out + i] instead (cols_out == cols_in).
-// Grids are at most 8 CTAs of 256 threads per SM (num_sms: the device's SM count).
+// out[i * ld_out + j] = bf16(scale * in[i * ld_in + j]) for j < cols_in, 0 for
+// cols_in <= j < cols_out (i < rows): the decode backward's split-K dX.  The
+// grid is at most 8 CTAs of 256 threads per SM (num_sms: the device's SM count).
 cudaError_t launch_convert_bf16(const float* in, int64_t rows, int64_t cols_in, int64_t ld_in,
                                 int64_t cols_out, float scale, uint16_t* out, int64_t ld_out, int num_sms,
                                 cudaStream_t stream);
-cudaError_t launch_convert_f32(const float* in, int64_t rows, int64_t cols, int64_t ld_in, float scale,
-                               bool transpose, float* out, int64_t ld_out, int num_sms, cudaStream_t stream);
 
 // LoRA gradients for few tokens (M <= 16), fp32 throughout on CUDA cores:
 //   dA[j, k] = s * sum_m G[m, j] X[m, k];   dB[n, j] = s * sum_m dY[m, n] XA[m, j]

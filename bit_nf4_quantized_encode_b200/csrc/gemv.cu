@@ -15,6 +15,7 @@
 //     [256 rows x 128 bytes] code tile (128B-swizzled) and the four [m x 64]
 //     activation boxes of each step into a 3- or 4-deep ring (TMA), and the
 //     warps write the step's block constants c1' = fma(e4m3(q), c2/448, mu)
+//     (or, for a weight stored without double quantization, its fp32 c1)
 //     into the stage.
 //   * Eight consumer warps own 32 weight rows each.  For every 64-column block
 //     they read their rows' code bytes, turn each byte into the two bf16 levels
@@ -162,13 +163,14 @@ __device__ __forceinline__ int64_t owner_of(int64_t u, int64_t total, int ctas) 
   return ((u + 1) * ctas - 1) / total;
 }
 
-// Block-constant inputs of one step for one weight row, loaded ahead: the E4M3
-// bytes of the step's four blocks (byte b = block b) and c2 of the first
-// block's group (and, when K is not a multiple of 256 columns, of the last
-// block's group too).
+// Block-constant inputs of one step for one weight row, loaded ahead.  With
+// double quantization: the E4M3 bytes of the step's four blocks (byte b =
+// block b) in q, and in v[0] c2 of the first block's group (in v[1], when K is
+// not a multiple of 256 columns, that of the last block's group too).
+// Without it: the four blocks' fp32 constants in v[0..3].
 struct RowConsts {
   uint32_t q;
-  float c2a, c2b;
+  float v[4];
 };
 
 // Eight consumer warps own 32 weight rows each (two m16 MMA tiles); warps
@@ -256,26 +258,37 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
     const bool tma_thread = hw == 0 && lane == 0;
     named_barrier_sync(2, kProducerWarps * 32);   // barrier initialisation seen by all producers
     named_barrier_arrive(1, kGemvThreads);
-    const float mu = __ldg(a.mean);
+    const float mu = a.absf != nullptr ? 0.0f : __ldg(a.mean);
+    const bool plain = a.absf != nullptr;
     auto load_raw = [&](Pos p, bool valid, RowConsts (&k)[kRowsPerProducerLane]) {
 #pragma unroll
       for (int j = 0; j < kRowsPerProducerLane; ++j) {
         k[j].q = 0;
-        k[j].c2a = 0.0f;
-        k[j].c2b = 0.0f;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) k[j].v[b] = 0.0f;
         const int64_t row = static_cast<int64_t>(p.tile) * kRows + 64 * hw + lane + 32 * j;
         if (valid && row < a.nw) {
           const uint32_t blk0 = static_cast<uint32_t>(row) * kbl + 4u * static_cast<uint32_t>(p.step);
-          if (kQuad) {
+          if (plain) {
+            if (kQuad) {           // blk0 is a multiple of 4: one 16-byte load
+              const float4 f = __ldg(reinterpret_cast<const float4*>(a.absf + blk0));
+              k[j].v[0] = f.x; k[j].v[1] = f.y; k[j].v[2] = f.z; k[j].v[3] = f.w;
+            } else {
+              const int nb = min(4, kblocks - 4 * p.step);
+#pragma unroll
+              for (int b = 0; b < 4; ++b)
+                if (b < nb) k[j].v[b] = __ldg(a.absf + blk0 + b);
+            }
+          } else if (kQuad) {
             k[j].q = __ldg(reinterpret_cast<const uint32_t*>(a.qabs + blk0));
-            k[j].c2a = __ldg(a.c2 + (blk0 >> 8));
+            k[j].v[0] = __ldg(a.c2 + (blk0 >> 8));
           } else {
             const int nb = min(4, kblocks - 4 * p.step);
 #pragma unroll
             for (int b = 0; b < 4; ++b)
               if (b < nb) k[j].q |= static_cast<uint32_t>(__ldg(a.qabs + blk0 + b)) << (8 * b);
-            k[j].c2a = __ldg(a.c2 + (blk0 >> 8));
-            k[j].c2b = __ldg(a.c2 + ((blk0 + nb - 1) >> 8));
+            k[j].v[0] = __ldg(a.c2 + (blk0 >> 8));
+            k[j].v[1] = __ldg(a.c2 + ((blk0 + nb - 1) >> 8));
           }
         }
       }
@@ -292,21 +305,26 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
         const int64_t row = static_cast<int64_t>(p.tile) * kRows + 64 * hw + lane + 32 * j;
         const uint32_t blk0 = static_cast<uint32_t>(row) * kbl + 4u * static_cast<uint32_t>(p.step);
         const uint32_t grp = blk0 >> 8;
-        if (grp != grp_cache[j]) {
-          grp_cache[j] = grp;
-          c2q_cache[j] = __fdiv_rn(k[j].c2a, 448.0f);
-        }
-        float f[4];
-        e4m3x4_to_f32(k[j].q, f);
         float c[4];
-        if (kQuad) {
+        if (plain) {
 #pragma unroll
-          for (int b = 0; b < 4; ++b) c[b] = __fmaf_rn(f[b], c2q_cache[j], mu);
+          for (int b = 0; b < 4; ++b) c[b] = k[j].v[b];
         } else {
-          const float c2q_b = __fdiv_rn(k[j].c2b, 448.0f);
+          if (grp != grp_cache[j]) {
+            grp_cache[j] = grp;
+            c2q_cache[j] = __fdiv_rn(k[j].v[0], 448.0f);
+          }
+          float f[4];
+          e4m3x4_to_f32(k[j].q, f);
+          if (kQuad) {
 #pragma unroll
-          for (int b = 0; b < 4; ++b)
-            c[b] = __fmaf_rn(f[b], ((blk0 + b) >> 8) == grp ? c2q_cache[j] : c2q_b, mu);
+            for (int b = 0; b < 4; ++b) c[b] = __fmaf_rn(f[b], c2q_cache[j], mu);
+          } else {
+            const float c2q_b = __fdiv_rn(k[j].v[1], 448.0f);
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+              c[b] = __fmaf_rn(f[b], ((blk0 + b) >> 8) == grp ? c2q_cache[j] : c2q_b, mu);
+          }
         }
         const uint32_t r = static_cast<uint32_t>(64 * hw + lane + 32 * j);
         sts128(hole(32u * slot + (r >> 3), (r & 7u) * 16u), c[0], c[1], c[2], c[3]);
@@ -434,10 +452,12 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
       }
     }
   };
-  // Y rows of tile `tile` for this lane from its fp32 sums: add the LoRA
-  // up-projection s (X A^T) B^T with warp MMAs (A operand = rows of B, B operand
-  // = the staged bf16(s X A^T)) and store bf16.
-  auto finish = [&](int tile, float (&acc)[2][kNT][4]) {
+  // The LoRA up-projection s (X A^T) B^T of one adapter added to this lane's
+  // fp32 sums with warp MMAs: A operand = rows of that adapter's B (lb), B
+  // operand = the staged bf16(s X A^T) of the tokens `use` selects (the other
+  // tokens enter as zeros).
+  auto lora_pass = [&](int tile, const uint16_t* __restrict__ lb, const bool (&use)[kNT],
+                       float (&acc)[2][kNT][4]) {
     const int64_t row0 = static_cast<int64_t>(tile) * kRows + warp * 32 + pg;
     for (int grp = 0; grp < a.lora_steps; ++grp) {
       uint4 xs[kNT][2];
@@ -448,7 +468,7 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
           uint4 u;
           asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w)
                        : "r"(sxa_addr(8 * n + g, grp, 2 * t + hf)) : "memory");
-          xs[n][hf] = u;
+          xs[n][hf] = use[n] ? u : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
@@ -460,7 +480,7 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
             const int64_t row = row0 + 8 * (2 * i + h);
             const int col = grp * 64 + 16 * t + 8 * hf;
             bv[h][hf] = (row < a.nw && col < a.r)
-                            ? __ldg(reinterpret_cast<const uint4*>(a.lora_b + row * a.r + col))
+                            ? __ldg(reinterpret_cast<const uint4*>(lb + row * a.r + col))
                             : make_uint4(0u, 0u, 0u, 0u);
           }
 #pragma unroll
@@ -476,6 +496,39 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
             }
           }
       }
+    }
+  };
+  // The adapters of a call with per-token adapters, each once (in order of
+  // first use); fn(adapter) is called for each.  Warp-uniform: every lane
+  // reads the same indices.
+  auto for_each_adapter = [&](auto&& fn) {
+    for (int j = 0; j < m; ++j) {
+      const int aj = __ldg(a.adapter_idx + j);
+      if (aj < 0 || aj >= a.n_adapters) continue;
+      bool first = true;
+      for (int k2 = 0; k2 < j; ++k2) first = first && __ldg(a.adapter_idx + k2) != aj;
+      if (first) fn(aj);
+    }
+  };
+  // Y rows of tile `tile` for this lane from its fp32 sums: add the LoRA term
+  // (one pass per adapter in use) and store bf16.
+  auto finish = [&](int tile, float (&acc)[2][kNT][4]) {
+    const int64_t row0 = static_cast<int64_t>(tile) * kRows + warp * 32 + pg;
+    if (a.adapter_idx == nullptr) {
+      bool all[kNT];
+#pragma unroll
+      for (int n = 0; n < kNT; ++n) all[n] = true;
+      lora_pass(tile, a.lora_b, all, acc);
+    } else {
+      int tok_ad[kNT];                              // the adapter of this lane's token 8n + g
+#pragma unroll
+      for (int n = 0; n < kNT; ++n) tok_ad[n] = 8 * n + g < m ? __ldg(a.adapter_idx + 8 * n + g) : -1;
+      for_each_adapter([&](int ad) {
+        bool use[kNT];
+#pragma unroll
+        for (int n = 0; n < kNT; ++n) use[n] = tok_ad[n] == ad;
+        lora_pass(tile, a.lora_b + static_cast<int64_t>(ad) * a.b_stride, use, acc);
+      });
     }
 #pragma unroll
     for (int i = 0; i < 2; ++i)
@@ -565,9 +618,13 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
   // group t of its rows, one 128-byte line per 64 rank columns)
   auto prefetch_b = [&](int tile) {
     const int64_t row = static_cast<int64_t>(tile) * kRows + warp * 32 + 8 * t + pg;
-    if (row < a.nw)
+    if (row >= a.nw) return;
+    auto rows_of = [&](const uint16_t* lb) {
       for (int grp = 0; grp < a.lora_steps; ++grp)
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(a.lora_b + row * a.r + grp * 64));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(lb + row * a.r + grp * 64));
+    };
+    if (a.adapter_idx == nullptr) rows_of(a.lora_b);
+    else for_each_adapter([&](int ad) { rows_of(a.lora_b + static_cast<int64_t>(ad) * a.b_stride); });
   };
 
   float y[2][kNT][4];
@@ -688,10 +745,25 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
 // 8-column chunks a block stride apart; the CTA reduces with warp shuffles and
 // one exchange through shared memory.  k_gemv, launched as the programmatic
 // dependent of this grid, waits for it only before it first counts a tile.
-template <int kMaxM>
+// The four A rows' 8 columns of chunk ch, unpacked.
+__device__ __forceinline__ void load_a_rows(const uint16_t* __restrict__ A, int j0, int r, int64_t kw,
+                                            int64_t ch, float (&af)[4][8]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 v = (j0 + c < r) ? __ldg(reinterpret_cast<const uint4*>(A + (j0 + c) * kw) + ch)
+                                 : make_uint4(0u, 0u, 0u, 0u);
+    af[c][0] = bf16_lo(v.x); af[c][1] = bf16_hi(v.x); af[c][2] = bf16_lo(v.y); af[c][3] = bf16_hi(v.y);
+    af[c][4] = bf16_lo(v.z); af[c][5] = bf16_hi(v.z); af[c][6] = bf16_lo(v.w); af[c][7] = bf16_hi(v.w);
+  }
+}
+
+// kMulti: every token has its own adapter (A + idx[i] * a_stride); its A rows
+// are loaded per token.  Tokens without a valid adapter accumulate nothing.
+template <int kMaxM, bool kMulti>
 __global__ void __launch_bounds__(64, 8)
 k_xa_zero(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A, int64_t m, int64_t kw, int r,
-          float* __restrict__ part, int64_t ld, float4* __restrict__ zero4, int64_t n4) {
+          float* __restrict__ part, int64_t ld, float4* __restrict__ zero4, int64_t n4,
+          const int32_t* __restrict__ idx, int n_adapters, int64_t a_stride, uint32_t* err) {
   launch_dependents();
   __shared__ float s_red[4 * kMaxM];
   const int mi = static_cast<int>(m);
@@ -703,21 +775,29 @@ k_xa_zero(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A, int64_
   for (int c = 0; c < 4; ++c)
 #pragma unroll
     for (int i = 0; i < kMaxM; ++i) acc[c][i] = 0.0f;
-  for (int64_t ch = c_beg + threadIdx.x; ch < c_end; ch += blockDim.x) {
-    float af[4][8];                        // the four A rows' 8 columns, unpacked once
+  int ad[kMaxM];                           // kMulti: token i's adapter, -1 for none
+  if constexpr (kMulti) {
+    bool bad = false;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint4 v = (j0 + c < r) ? __ldg(reinterpret_cast<const uint4*>(A + (j0 + c) * kw) + ch)
-                                   : make_uint4(0u, 0u, 0u, 0u);
-      af[c][0] = bf16_lo(v.x); af[c][1] = bf16_hi(v.x); af[c][2] = bf16_lo(v.y); af[c][3] = bf16_hi(v.y);
-      af[c][4] = bf16_lo(v.z); af[c][5] = bf16_hi(v.z); af[c][6] = bf16_lo(v.w); af[c][7] = bf16_hi(v.w);
+    for (int i = 0; i < kMaxM; ++i) {
+      ad[i] = i < mi ? __ldg(idx + i) : -1;
+      if (ad[i] >= n_adapters) { bad = true; ad[i] = -1; }
     }
+    if (bad && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) atomicOr(err, kErrBadAdapter);
+  }
+  for (int64_t ch = c_beg + threadIdx.x; ch < c_end; ch += blockDim.x) {
+    float af[4][8];
+    if constexpr (!kMulti) load_a_rows(A, j0, r, kw, ch, af);   // shared by every token
     uint4 xv[kMaxM];
 #pragma unroll
     for (int i = 0; i < kMaxM; ++i)
       xv[i] = i < mi ? __ldg(reinterpret_cast<const uint4*>(X + i * kw) + ch) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
     for (int i = 0; i < kMaxM; ++i) {
+      if constexpr (kMulti) {
+        if (ad[i] < 0) continue;
+        load_a_rows(A + static_cast<int64_t>(ad[i]) * a_stride, j0, r, kw, ch, af);
+      }
       const float xf[8] = {bf16_lo(xv[i].x), bf16_hi(xv[i].x), bf16_lo(xv[i].y), bf16_hi(xv[i].y),
                            bf16_lo(xv[i].z), bf16_hi(xv[i].z), bf16_lo(xv[i].w), bf16_hi(xv[i].w)};
 #pragma unroll
@@ -808,15 +888,26 @@ int64_t gemv_slot_floats(int64_t m_tiles, int64_t steps) {
   return ctas * 2 * kConsumerWarps * 32 * 16;
 }
 
+template <bool kMulti>
+void launch_xa_zero_t(dim3 grid, const uint16_t* X, const uint16_t* A, int64_t m, int64_t kw, int r,
+                      float* part, int64_t ld, float4* z4, int64_t n4, const int32_t* idx, int n_ad,
+                      int64_t a_stride, uint32_t* err, cudaStream_t stream) {
+  if (m <= 1) k_xa_zero<1, kMulti><<<grid, 64, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4, idx, n_ad, a_stride, err);
+  else if (m <= 4) k_xa_zero<4, kMulti><<<grid, 64, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4, idx, n_ad, a_stride, err);
+  else if (m <= 8) k_xa_zero<8, kMulti><<<grid, 64, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4, idx, n_ad, a_stride, err);
+  else k_xa_zero<16, kMulti><<<grid, 64, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4, idx, n_ad, a_stride, err);
+}
+
 cudaError_t launch_xa_zero(const uint16_t* X, const uint16_t* A, int64_t m, int64_t kw, int r, float* part,
-                           int64_t ld, int splits, float* zero, int64_t n_zero, cudaStream_t stream) {
+                           int64_t ld, int splits, float* zero, int64_t n_zero, const int32_t* adapter_idx,
+                           int n_adapters, int64_t a_stride, uint32_t* err, cudaStream_t stream) {
   const dim3 grid(static_cast<unsigned>((r + 3) / 4), static_cast<unsigned>(splits));
   float4* z4 = reinterpret_cast<float4*>(zero);
   const int64_t n4 = n_zero / 4;
-  if (m <= 1) k_xa_zero<1><<<grid, 64, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4);
-  else if (m <= 4) k_xa_zero<4><<<grid, 64, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4);
-  else if (m <= 8) k_xa_zero<8><<<grid, 64, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4);
-  else k_xa_zero<16><<<grid, 64, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4);
+  if (adapter_idx)
+    launch_xa_zero_t<true>(grid, X, A, m, kw, r, part, ld, z4, n4, adapter_idx, n_adapters, a_stride, err, stream);
+  else
+    launch_xa_zero_t<false>(grid, X, A, m, kw, r, part, ld, z4, n4, nullptr, 1, 0, err, stream);
   return cudaGetLastError();
 }
 

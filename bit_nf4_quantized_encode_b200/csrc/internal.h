@@ -4,6 +4,8 @@
 #pragma once
 #include <cuda_runtime.h>
 
+#include "codec.h"
+#include "nf4_tables.h"
 #include "qlora.h"
 
 namespace qlora {
@@ -16,6 +18,9 @@ cudaError_t counted(cudaError_t e, int n = 1);
 // shape range (0 <= rows, cols <= 2^31), block sizes, then (for a non-empty
 // weight) NULL buffers and 16-byte alignment, in that order.
 qlora_status check_tensor(const qlora_nf4_tensor* t);
+
+// The encode kernel's bucket tables (kernel parameter) of one type's tables.
+EncodeTables encode_tables(const Nf4Tables& tabs);
 
 // Device address of the library's error flag on the current device (the flag
 // qlora_read_device_errors reads); QLORA_ERR_UNSUPPORTED on a non-sm_100 device.

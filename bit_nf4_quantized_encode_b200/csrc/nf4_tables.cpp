@@ -4,7 +4,12 @@
 // explained", paragraph "4-bit NormalFloat (NF4)": levels at the quantiles of
 // a standard normal; creativeworksofknowledge "QLoRA: Fine-Tune 70B on One
 // GPU", section "1. NF4": Gaussian-proportional levels, denser near zero).
-// Construction: 8 positive levels at Phi^-1(1/2 + (delta - 1/2) j / 8),
+// The comparison types of automatone, "4-bit NormalFloat (NF4)" (evenly spaced
+// 4-bit integers, exponent-spaced 4-bit floats) get tables of their own: INT4
+// levels (2i - 15) / 15, and FP4 the E2M1 values divided by 6 (15 distinct
+// values; the last code repeats +1).
+//
+// NF4 construction: 8 positive levels at Phi^-1(1/2 + (delta - 1/2) j / 8),
 // j = 1..8, 7 negative levels at -Phi^-1(1/2 + (delta - 1/2) j / 7), j = 1..7,
 // and an exact zero, all divided by Phi^-1(delta), with
 // delta = 1 - (1/30 + 1/32) / 2; evaluated in double and rounded once to float.
@@ -66,15 +71,36 @@ float from_key(uint32_t k) {
   return f;
 }
 
-Nf4Tables build() {
+// The 16 levels of each 4-bit type, ascending, in [-1, 1].
+void make_levels(int type, float (&level)[16]) {
+  if (type == kTypeNf4) {
+    const double delta = 1.0 - 0.5 * (1.0 / 30.0 + 1.0 / 32.0);
+    const double top = inv_normal_cdf(delta);
+    for (int j = 1; j <= 7; ++j)
+      level[7 - j] = static_cast<float>(-inv_normal_cdf(0.5 + (delta - 0.5) * j / 7.0) / top);
+    level[7] = 0.0f;
+    for (int j = 1; j <= 8; ++j)
+      level[7 + j] = static_cast<float>(inv_normal_cdf(0.5 + (delta - 0.5) * j / 8.0) / top);
+  } else if (type == kTypeInt4) {
+    // 16 evenly spaced integers -15, -13, ..., 15 over the half-range 15
+    for (int i = 0; i < 16; ++i) level[i] = static_cast<float>(static_cast<double>(2 * i - 15) / 15.0);
+  } else {
+    // E2M1: magnitudes m * 2^-1 (exponent field 0) and (1 + m/2) * 2^(e - 1);
+    // the 8 non-negative ones ascending are the table's upper half from index 7
+    double mag[8];
+    int k = 0;
+    for (int e = 0; e < 4; ++e)
+      for (int m = 0; m < 2; ++m) mag[k++] = e == 0 ? 0.5 * m : std::ldexp(1.0 + 0.5 * m, e - 1);
+    const double top = mag[7];
+    for (int i = 0; i < 8; ++i) level[7 + i] = static_cast<float>(mag[i] / top);
+    for (int i = 1; i < 8; ++i) level[7 - i] = static_cast<float>(-mag[i] / top);   // -0 is the same level as +0
+    level[15] = level[14];    // 15 distinct values: the last code repeats +1 and is never chosen
+  }
+}
+
+Nf4Tables build(int type) {
   Nf4Tables t{};
-  const double delta = 1.0 - 0.5 * (1.0 / 30.0 + 1.0 / 32.0);
-  const double top = inv_normal_cdf(delta);
-  for (int j = 1; j <= 7; ++j)
-    t.level[7 - j] = static_cast<float>(-inv_normal_cdf(0.5 + (delta - 0.5) * j / 7.0) / top);
-  t.level[7] = 0.0f;
-  for (int j = 1; j <= 8; ++j)
-    t.level[7 + j] = static_cast<float>(inv_normal_cdf(0.5 + (delta - 0.5) * j / 8.0) / top);
+  make_levels(type, t.level);
 
   // Nearest level with ties to the lower index <=> count of thresholds <= n,
   // where threshold i is the first float past the midpoint of levels i, i+1.
@@ -128,11 +154,15 @@ Nf4Tables build() {
 
 }  // namespace
 
-const Nf4Tables& nf4_tables() {
-  static Nf4Tables tables;
+const Nf4Tables& level_tables(int type) {
+  static Nf4Tables tables[kNumTypes];
   static std::once_flag once;
-  std::call_once(once, [] { tables = build(); });
-  return tables;
+  std::call_once(once, [] {
+    for (int i = 0; i < kNumTypes; ++i) tables[i] = build(i);
+  });
+  return tables[(type >= 0 && type < kNumTypes) ? type : kTypeNf4];
 }
+
+const Nf4Tables& nf4_tables() { return level_tables(kTypeNf4); }
 
 }  // namespace qlora

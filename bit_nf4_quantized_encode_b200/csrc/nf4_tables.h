@@ -10,7 +10,7 @@ namespace qlora {
 constexpr int kNumBuckets = 33;
 
 struct Nf4Tables {
-  float level[16];            // NF4 levels, ascending, level[7] == 0
+  float level[16];            // levels, ascending (FP4 repeats +1 in the last entry)
   float threshold[15];        // code(n) = #{i : n >= threshold[i]}
   float bucket_thr[kNumBuckets];     // the one threshold inside bucket u, or +inf
   uint8_t bucket_base[kNumBuckets];  // code of the smallest n in bucket u
@@ -22,7 +22,15 @@ struct Nf4Tables {
   bool fast_ok;               // every threshold lies more than 2^-18 inside its bucket
 };
 
-// Built once (thread-safe) on first use.
+// The 4-bit data types: the values of qlora_nf4_tensor::quant_type.
+constexpr int kTypeNf4 = 0;
+constexpr int kTypeFp4 = 1;
+constexpr int kTypeInt4 = 2;
+constexpr int kNumTypes = 3;
+
+// The tables of one type (NF4 for an unknown type), all built once
+// (thread-safe) on first use.
+const Nf4Tables& level_tables(int type);
 const Nf4Tables& nf4_tables();
 
 }  // namespace qlora

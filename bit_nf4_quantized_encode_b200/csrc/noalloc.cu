@@ -83,23 +83,18 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const uint16_t* W, const q
   if ((reinterpret_cast<uintptr_t>(W) & 15u) != 0) return QLORA_ERR_ALIGN;
   // in place of the work-buffer size check: the built-in scratch's limit
   if (numel > QLORA_NOALLOC_MAX_ELEMENTS) return QLORA_ERR_WORKSPACE;
-  const Nf4Tables& tabs = nf4_tables();
+  const Nf4Tables& tabs = level_tables(out->quant_type);
   if (!tabs.ok) return QLORA_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   int num_sms = 0;
   st = scratch_for_current_device(&scratch, &num_sms);
   if (st != QLORA_OK) return st;
-
-  EncodeTables et;
-  for (int i = 0; i < kBuckets; ++i) {
-    et.bucket_thr[i] = i < kNumBuckets ? tabs.bucket_thr[i] : INFINITY;
-    et.bucket_base[i] = i < kNumBuckets ? tabs.bucket_base[i] : 15;
-    et.bucket_fast[i] = i < kNumBuckets ? tabs.bucket_fast[i] : (0x7F7FFFE0u | 16u);
-  }
-  et.fast = tabs.fast_ok ? 1 : 0;
+  const EncodeTables et = encode_tables(tabs);
+  const bool dq = out->blocksize2 != 0;
 
   const int64_t nblocks = (numel + 63) / 64;
-  float* c1buf = static_cast<float*>(scratch);
+  // without double quantization the block absmax values are the output itself
+  float* c1buf = dq ? static_cast<float*>(scratch) : out->absmax;
   double* partials = reinterpret_cast<double*>(static_cast<unsigned char*>(scratch) + kNoAllocC1Bytes);
   int grid = static_cast<int>((nblocks * 8 + 255) / 256);
   const int wave = num_sms * encode_ctas_per_sm();             // one wave of resident CTAs
@@ -108,6 +103,7 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const uint16_t* W, const q
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (counted(launch_encode(W, numel, et, out->codes, c1buf, partials, grid, s)) != cudaSuccess)
     return QLORA_ERR_CUDA;
+  if (!dq) return QLORA_OK;
   const int64_t ngroups = (nblocks + 255) / 256;
   int grid2 = static_cast<int>((ngroups + 7) / 8);
   if (grid2 > num_sms * 4) grid2 = num_sms * 4;

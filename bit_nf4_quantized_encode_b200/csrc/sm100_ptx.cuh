@@ -16,6 +16,7 @@ enum : uint32_t {
   kErrWaitTimeout = 1u << 0,   // an mbarrier wait gave up
   kErrTmemAlloc   = 1u << 1,   // TMEM allocation returned an unexpected address
   kErrSmemLayout  = 1u << 2,   // the shared-memory window does not fit a kernel's fixed map
+  kErrBadAdapter  = 1u << 3,   // a per-token adapter index is not in the adapter stack
 };
 
 // Bound on any single mbarrier wait, in SM clock cycles (about two seconds at

@@ -33,10 +33,11 @@
  *   - Thread safety: calls may be made concurrently on different streams;
  *     calls sharing a work buffer must be ordered by the caller.
  *   - Reproducibility: NF4 codes, E4M3 constants, c2, the mean and the
- *     dequantized weight are bit-exact and deterministic.  Results that sum
- *     split-K partials with fp32 atomics can differ in the last bits from run
- *     to run (the order of the additions varies): the saved X A^T, dA and dB
- *     with more than 16 tokens, and dX with 16 tokens or fewer.
+ *     dequantized weight are bit-exact and deterministic.  Y, X A^T, dA, dB
+ *     and (with more than 16 tokens) dX are bit-reproducible from run to run
+ *     on the same device: split contractions sum their partials in a fixed
+ *     order.  The one exception is dX with 16 tokens or fewer, whose split-K
+ *     partials are added with fp32 atomics and can differ in the last bits.
  */
 #ifndef QLORA_H_
 #define QLORA_H_
@@ -61,23 +62,44 @@ typedef enum {
   QLORA_ERR_NULL = -1,         /* a required pointer is NULL */
   QLORA_ERR_SHAPE = -2,        /* a size is out of range or not a supported multiple */
   QLORA_ERR_ALIGN = -3,        /* a pointer is not 16-byte aligned */
-  QLORA_ERR_UNSUPPORTED = -4,  /* block sizes other than 64 / 256, or no sm_100 device */
+  QLORA_ERR_UNSUPPORTED = -4,  /* block sizes, quant type, or no sm_100 device */
   QLORA_ERR_CUDA = -5,         /* a CUDA runtime / driver call failed */
   QLORA_ERR_WORKSPACE = -6     /* the work buffer is smaller than required */
 } qlora_status;
+
+/*
+ * The 4-bit data type of a quantized weight (its 16 levels, ascending, in
+ * [-1, 1]; qlora_get_levels returns them).  NF4 is the method's type
+ * (automatone "QLoRA paper explained", paragraph "4-bit NormalFloat (NF4)");
+ * INT4 and FP4 are the types that paragraph compares it with:
+ *   QLORA_NF4   normal quantiles with an exact zero at index 7 (see
+ *               qlora_get_codebook);
+ *   QLORA_FP4   the E2M1 4-bit float values divided by 6: 15 distinct levels
+ *               (+0 and -0 are one), index 7 is 0, the last entry repeats +1
+ *               and is never chosen by the encoder;
+ *   QLORA_INT4  16 evenly spaced levels (2i - 15) / 15 (no exact zero).
+ */
+typedef enum { QLORA_NF4 = 0, QLORA_FP4 = 1, QLORA_INT4 = 2 } qlora_quant_type;
 
 /*
  * A quantized weight W [rows, cols] (rows = out features N, cols = in
  * features K).  Layout of the flattened row-major weight e = n*cols + k:
  *   codes      [ceil(rows*cols/2)] bytes; byte j holds element 2j in its high
  *              nibble and element 2j+1 in its low nibble; a ragged tail is
- *              padded with code 7 (the zero level).
- *   absmax_q   [ceil(rows*cols/64)] OCP E4M3 codes, one per 64-weight block.
- *   absmax_c2  [ceil(ceil(rows*cols/64)/256)] float, one per 256 blocks.
- *   absmax_mean[1] float, the mean of all block absmax values.
- * Dequantized weight: c1' = fma(e4m3(q[b]), c2[b/256] / 448, mean);
- *                     w'  = bf16_RNE(L[code] * c1').
- * All four buffers are caller-owned device memory.
+ *              padded with code 7; a block whose absmax is 0 is all code 7.
+ * The block constants, one per 64 weights, are stored in one of two forms:
+ *   with double quantization (blocksize2 = 256; creativeworksofknowledge
+ *   "QLoRA: Fine-Tune 70B on One GPU", "2. Double quantization"):
+ *     absmax_q   [ceil(rows*cols/64)] OCP E4M3 codes, one per 64-weight block.
+ *     absmax_c2  [ceil(ceil(rows*cols/64)/256)] float, one per 256 blocks.
+ *     absmax_mean[1] float, the mean of all block absmax values.
+ *     Dequantized weight: c1' = fma(e4m3(q[b]), c2[b/256] / 448, mean);
+ *                         w'  = bf16_RNE(L[code] * c1').
+ *   without it (blocksize2 = 0, 0.5 bits of constants per weight):
+ *     absmax     [ceil(rows*cols/64)] float, the block absmax c1 itself.
+ *     Dequantized weight: w' = bf16_RNE(L[code] * c1).
+ * Pointers of the form not in use are ignored (may be NULL).  All buffers are
+ * caller-owned device memory.  A zero-initialised quant_type is NF4.
  */
 typedef struct {
   uint8_t* codes;
@@ -87,7 +109,10 @@ typedef struct {
   int64_t rows;
   int64_t cols;
   int32_t blocksize;    /* must be 64 */
-  int32_t blocksize2;   /* must be 256 */
+  int32_t blocksize2;   /* 256: double quantization; 0: fp32 block constants */
+  float* absmax;        /* blocksize2 == 0 only */
+  int32_t quant_type;   /* a qlora_quant_type */
+  int32_t reserved;     /* must be 0 */
 } qlora_nf4_tensor;
 
 /* Human-readable name of a status. Never NULL. */
@@ -102,8 +127,16 @@ QLORA_EXPORT const char* qlora_status_string(qlora_status s);
 QLORA_EXPORT void qlora_get_codebook(float out[16]);
 
 /*
+ * The 16 levels of a 4-bit type (see qlora_quant_type).  Host only.
+ * Errors: QLORA_ERR_NULL, QLORA_ERR_UNSUPPORTED (unknown type).
+ */
+QLORA_EXPORT qlora_status qlora_get_levels(int32_t quant_type, float out[16]);
+
+/*
  * Byte sizes of the buffers of a quantized [rows, cols] weight and of the
  * work buffer qlora_quantize_nf4_dq needs.  Any output pointer may be NULL.
+ * With blocksize2 = 0 (no double quantization) absmax_q_bytes receives the
+ * size of the fp32 `absmax` array and absmax_c2_bytes 0.
  * Errors: QLORA_ERR_SHAPE (rows or cols < 0), QLORA_ERR_UNSUPPORTED (block sizes).
  */
 QLORA_EXPORT qlora_status qlora_nf4_sizes(int64_t rows, int64_t cols, int32_t blocksize, int32_t blocksize2,
@@ -111,13 +144,16 @@ QLORA_EXPORT qlora_status qlora_nf4_sizes(int64_t rows, int64_t cols, int32_t bl
                              size_t* workspace_bytes);
 
 /*
- * Blockwise absmax NF4 encode of a bf16 weight, then double quantization of
- * the block constants (automatone, "4-bit NormalFloat (NF4)" and "Double
- * Quantization (DQ)"; creativeworksofknowledge, "2. Double quantization"):
+ * Blockwise absmax encode of a bf16 weight with the levels of
+ * out->quant_type, then double quantization of the block constants
+ * (automatone, "4-bit NormalFloat (NF4)" and "Double Quantization (DQ)";
+ * creativeworksofknowledge, "2. Double quantization"):
  *   per 64 weights: c1 = max|x|, n = x / c1 (IEEE), code = nearest level
  *   (ties to the lower index); per tensor: mean = float(sum(c1) / count)
  *   with the sum in double; per 256 constants: c2 = max|c1 - mean|,
  *   q = E4M3_RNE(float((c1 - mean) / c2) * 448), q = 0 when c2 == 0.
+ * With out->blocksize2 == 0 the constants c1 are written to out->absmax as
+ * they are (no double quantization).
  * W: [out->rows * out->cols] bf16.  out: the destination buffers and shape.
  * workspace: >= workspace_bytes of qlora_nf4_sizes.
  * A zero-sized weight is a no-op.
@@ -126,8 +162,9 @@ QLORA_EXPORT qlora_status qlora_quantize_nf4_dq(const uint16_t* W, const qlora_n
                                    size_t workspace_bytes, qlora_stream_t stream);
 
 /*
- * Two-level dequantization to bf16 (automatone "How it works": dequantize to
- * the BFloat16 compute type).  W_out: [rows * cols] bf16.
+ * Dequantization to bf16 (automatone "How it works": dequantize to the
+ * BFloat16 compute type): two-level with double quantization, one fp32
+ * constant per block without it (see qlora_nf4_tensor).  W_out: [rows * cols] bf16.
  */
 QLORA_EXPORT qlora_status qlora_dequantize(const qlora_nf4_tensor* W, uint16_t* W_out, qlora_stream_t stream);
 
@@ -157,6 +194,28 @@ QLORA_EXPORT qlora_status qlora_linear_fwd(const qlora_nf4_tensor* W, const uint
                               qlora_stream_t stream);
 
 /*
+ * Decode-shaped forward with a LoRA adapter per token: several adapters served
+ * over one frozen 4-bit weight in one pass over it (automatone "QLoRA paper
+ * explained", "Results": the 4-bit base is also the deployed model).  Token t
+ * uses adapter a = adapter_idx[t]:
+ *   Y[t] = X[t] deq(W)^T + s (X[t] A_a^T) B_a^T,   XA_out[t] = X[t] A_a^T
+ * A_stack [n_adapters][r, cols] bf16 and B_stack [n_adapters][rows, r] bf16,
+ * each adapter contiguous; adapter_idx: device int32 [M], 4-byte aligned.  A
+ * negative index means "no adapter" (the base weight alone, XA_out row 0).
+ * An index >= n_adapters is treated the same way and sets bit 3 of the device
+ * error flag (qlora_read_device_errors): it cannot be checked on the host.
+ * The weight is read once whatever the number of adapters; every adapter in
+ * use adds one rank-r up-projection per output tile.
+ * Requirements as qlora_linear_fwd, and 1 <= M <= 16, n_adapters >= 1; the
+ * work buffer is qlora_linear_workspace_size's fwd_bytes for the same M.
+ */
+QLORA_EXPORT qlora_status qlora_linear_fwd_multi(const qlora_nf4_tensor* W, const uint16_t* X, int64_t M,
+                                    const uint16_t* A_stack, const uint16_t* B_stack, int32_t n_adapters,
+                                    const int32_t* adapter_idx, int32_t r, float s, uint16_t* Y,
+                                    float* XA_out, void* workspace, size_t workspace_bytes,
+                                    qlora_stream_t stream);
+
+/*
  * Backward of the same layer; W is frozen and gets no gradient (automatone
  * "How it works": gradients land only on the LoRA adapters; gptget Deep
  * Analysis: backward dequantizes to 16-bit for the matmul):
@@ -177,7 +236,10 @@ QLORA_EXPORT qlora_status qlora_linear_bwd(const qlora_nf4_tensor* W, const uint
 /*
  * Device error flag of the calling thread's current device: bit 0 is set when
  * a kernel's internal wait gave up after its time limit (a bug, reported
- * instead of hanging).  Reading synchronizes the device; clear = 1 resets it.
+ * instead of hanging); bit 2 when a kernel's shared-memory window did not fit
+ * its fixed map; bit 3 when a per-token adapter index was out of range
+ * (qlora_linear_fwd_multi).  Reading synchronizes the device; clear = 1
+ * resets it.
  */
 QLORA_EXPORT qlora_status qlora_read_device_errors(uint32_t* flags, int clear);
 

@@ -100,6 +100,10 @@ def _load():
         lib.nf4o_bf16_rne_n.restype = None
         lib.nf4o_e4m3_rne_n.argtypes = [f32p, i64, u8p]
         lib.nf4o_e4m3_rne_n.restype = None
+        lib.nf4o_levels.argtypes = [ctypes.c_int, f32p]
+        lib.nf4o_levels.restype = ctypes.c_int
+        lib.nf4o_dequant_f32.argtypes = [u8p, f32p, i64, ctypes.c_int, f32p, u16p]
+        lib.nf4o_dequant_f32.restype = None
         _lib = lib
         return lib
 
@@ -171,6 +175,22 @@ def codebook(delta: float | None = None) -> np.ndarray:
     return out
 
 
+# The 4-bit data types (reading R7): NF4, and the two the pages compare it with
+# (automatone "QLoRA paper explained", "4-bit NormalFloat (NF4)": evenly spaced
+# 4-bit integers, exponent-spaced 4-bit floats).
+QUANT_TYPES = {"nf4": 0, "fp4": 1, "int4": 2}
+
+
+def levels(quant_type: str = "nf4") -> np.ndarray:
+    """The 16 levels of a 4-bit data type as float32, ascending, in [-1, 1]:
+    NF4 (the codebook above), INT4 ((2i - 15) / 15) or FP4 (the 15 distinct
+    E2M1 values / 6, then +1 repeated; code 15 is never chosen)."""
+    out = np.zeros(16, dtype=np.float32)
+    if _load().nf4o_levels(QUANT_TYPES[quant_type], _ptr(out, ctypes.c_float)) != 0:
+        raise ValueError(quant_type)
+    return out
+
+
 def nearest(n: float, L: np.ndarray | None = None) -> int:
     if L is None:
         L = codebook()
@@ -183,7 +203,9 @@ def nearest(n: float, L: np.ndarray | None = None) -> int:
 # ---------------------------------------------------------------------------
 
 def storage_bytes(numel: int, bs: int = BLOCKSIZE, bs2: int = BLOCKSIZE2) -> dict:
-    """Bytes of each buffer of a quantized tensor with `numel` weights."""
+    """Bytes of each buffer of a quantized tensor with `numel` weights.  With
+    bs2 = 0 (no double quantization) 'absmax_q' is the fp32 absmax array and
+    there is no c2 or mean."""
     out = [ctypes.c_int64() for _ in range(4)]
     _load().nf4o_storage_bytes(int(numel), int(bs), int(bs2), *[ctypes.byref(o) for o in out])
     return dict(codes=out[0].value, absmax_q=out[1].value, absmax_c2=out[2].value,
@@ -218,7 +240,7 @@ def block_mean(c1: np.ndarray) -> np.float32:
     return np.float32(_load().nf4o_mean(_ptr(c, ctypes.c_float), c.size))
 
 
-def double_quant(c1: np.ndarray, bs2: int = BLOCKSIZE2):
+def double_quant_fn(c1: np.ndarray, bs2: int = BLOCKSIZE2):
     """Returns (q uint8 [nblocks] E4M3 codes, c2 float32 [ngroups], mean float32)."""
     c = np.ascontiguousarray(c1, dtype=np.float32)
     nb = c.size
@@ -230,6 +252,9 @@ def double_quant(c1: np.ndarray, bs2: int = BLOCKSIZE2):
         _load().nf4o_double_quant(_ptr(c, ctypes.c_float), nb, bs2, _ptr(q, ctypes.c_uint8),
                                   _ptr(c2, ctypes.c_float), _ptr(mu, ctypes.c_float))
     return q[:nb], c2[:ng], mu[0]
+
+
+double_quant = double_quant_fn
 
 
 def block_constant(q: int, c2: float, mu: float) -> np.float32:
@@ -254,18 +279,52 @@ def dequant(packed, q, c2, mu, numel: int, bs: int = BLOCKSIZE, bs2: int = BLOCK
     return out[:numel]
 
 
-def quantize(w_bits: np.ndarray, bs: int = BLOCKSIZE, bs2: int = BLOCKSIZE2) -> dict:
-    """Encode then double-quantize: the full stored form of one weight tensor."""
-    packed, c1 = encode(w_bits, bs)
-    q, c2, mu = double_quant(c1, bs2)
-    return dict(codes=packed, absmax_q=q, absmax_c2=c2, mean=mu, c1=c1,
-                numel=int(np.asarray(w_bits).size), shape=tuple(np.asarray(w_bits).shape))
+def dequant_f32(packed, c1, numel: int, bs: int = BLOCKSIZE, L: np.ndarray | None = None) -> np.ndarray:
+    """Dequantization without double quantization: w' = bf16_RNE(L[code] * c1)
+    with the block's fp32 absmax c1; returns uint16 bit patterns [numel]."""
+    if L is None:
+        L = codebook()
+    p = np.ascontiguousarray(packed, dtype=np.uint8)
+    cc = np.ascontiguousarray(c1, dtype=np.float32)
+    Lc = np.ascontiguousarray(L, dtype=np.float32)
+    out = np.zeros(max(int(numel), 1), dtype=np.uint16)
+    if numel:
+        _load().nf4o_dequant_f32(_ptr(p, ctypes.c_uint8), _ptr(cc, ctypes.c_float), int(numel), bs,
+                                 _ptr(Lc, ctypes.c_float), _ptr(out, ctypes.c_uint16))
+    return out[:numel]
+
+
+def quantize(w_bits: np.ndarray, bs: int = BLOCKSIZE, bs2: int = BLOCKSIZE2, quant_type: str = "nf4",
+             double_quant: bool = True) -> dict:
+    """Encode (with the levels of `quant_type`), then double-quantize the block
+    constants -- or, with double_quant=False, keep them as fp32 (the variant
+    without double quantization).  The full stored form of one weight tensor."""
+    L = levels(quant_type)
+    packed, c1 = encode(w_bits, bs, L)
+    qt = dict(codes=packed, c1=c1, quant_type=quant_type, double_quant=double_quant, levels=L,
+              numel=int(np.asarray(w_bits).size), shape=tuple(np.asarray(w_bits).shape))
+    if double_quant:
+        q, c2, mu = double_quant_fn(c1, bs2)
+        qt.update(absmax_q=q, absmax_c2=c2, mean=mu)
+    else:
+        qt.update(absmax=c1.copy())
+    return qt
 
 
 def dequant_tensor(qt: dict, bs: int = BLOCKSIZE, bs2: int = BLOCKSIZE2) -> np.ndarray:
     """deq(W) as float32 values (bf16-exact), reshaped like the original weight."""
-    bits = dequant(qt["codes"], qt["absmax_q"], qt["absmax_c2"], qt["mean"], qt["numel"], bs, bs2)
+    bits = dequant_bits(qt, bs, bs2)
     return bf16_bits_to_f32(bits).reshape(qt["shape"])
+
+
+def dequant_bits(qt: dict, bs: int = BLOCKSIZE, bs2: int = BLOCKSIZE2) -> np.ndarray:
+    """deq(W) as bf16 bit patterns [numel], for either stored form."""
+    L = qt.get("levels")
+    if L is None:
+        L = codebook()
+    if qt.get("double_quant", True):
+        return dequant(qt["codes"], qt["absmax_q"], qt["absmax_c2"], qt["mean"], qt["numel"], bs, bs2, L)
+    return dequant_f32(qt["codes"], qt["absmax"], qt["numel"], bs, L)
 
 
 # ---------------------------------------------------------------------------
@@ -308,6 +367,26 @@ def lora_grads(X, dY, A, B, s: float):
     dA = s * (G.T @ X)
     dB = s * (dY.T @ XA)
     return XA, G, dA, dB
+
+
+def linear_fwd_multi(Wd, X, A_stack, B_stack, adapter_idx, s: float):
+    """Forward with a LoRA adapter per token (batched decode of several adapters
+    over one frozen weight; automatone "QLoRA paper explained", "Results": the
+    4-bit base is also what gets deployed).  Token t uses adapter
+    a = adapter_idx[t]:  Y[t] = X[t] W'^T + s (X[t] A_a^T) B_a^T  and
+    XA[t] = X[t] A_a^T; a token whose index is negative (or not in the stack)
+    gets no LoRA term and XA[t] = 0.  A_stack [n, r, K], B_stack [n, N, r].
+    Returns (Y, XA) in float64."""
+    Wd, X = _f64(Wd), _f64(X)
+    A_stack, B_stack = _f64(A_stack), _f64(B_stack)
+    n_ad, r = A_stack.shape[0], A_stack.shape[1]
+    Y = X @ Wd.T
+    XA = np.zeros((X.shape[0], r))
+    for t, a in enumerate(np.asarray(adapter_idx).reshape(-1)):
+        if 0 <= a < n_ad:
+            XA[t] = X[t] @ A_stack[a].T
+            Y[t] += s * (XA[t] @ B_stack[a].T)
+    return Y, XA
 
 
 def linear_fwd_rows(Wd, X, A, B, s: float, rows):

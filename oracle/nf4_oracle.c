@@ -42,6 +42,9 @@
  *       q = E4M3(RNE(float(float((c1 - mu) / c2) * 448))); q = 0 if c2 == 0.
  *       FP8 is OCP E4M3 "fn" (max 448, no infinities).
  *   R6  dequant: c1' = fmaf(e4m3(q), c2 / 448, mu); w' = bf16_RNE(L[code]*c1').
+ *       Without double quantization the constant is c1 itself (fp32).
+ *   R7  the comparison types INT4 and FP4 (see nf4o_levels); the encode,
+ *       packing and constants are the same for every type.
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fopenmp -fPIC
  * -shared.  FP contraction is off so every float operation rounds once, as
@@ -182,15 +185,87 @@ NF4O_EXPORT int nf4o_nearest(float n, const float L[16])
 }
 
 /* ---------------------------------------------------------------------- */
+/* R7: the other 4-bit data types the pages compare NF4 with.             */
+/* ---------------------------------------------------------------------- */
+
+/* automatone, "4-bit NormalFloat (NF4)": standard 4-bit integers space their
+ * 16 levels evenly, 4-bit floats space theirs by exponent, and NF4 beats both
+ * (also "Results": FP4 trails NF4).  Both tables are normalized to [-1, 1],
+ * the range blockwise absmax scaling maps a block into.
+ *
+ * INT4: 16 evenly spaced levels from -1 to +1, L[i] = (2i - 15) / 15 (no
+ *   exact zero: 16 even steps over a symmetric range cannot have one).
+ * FP4:  the values of the 4-bit float E2M1 (1 sign bit, 2 exponent bits with
+ *   bias 1, 1 mantissa bit; exponent field 0 is subnormal), decoded from each
+ *   of the 16 bit patterns and divided by the largest magnitude, 6.  +0 and -0
+ *   are one value, so there are 15 distinct levels: they fill L[0..14] in
+ *   ascending order and L[15] repeats +1.  Code 15 is never chosen: the
+ *   nearest-level rule sends a tie to the lower index. */
+#define NF4O_TYPE_NF4 0
+#define NF4O_TYPE_FP4 1
+#define NF4O_TYPE_INT4 2
+
+static double e2m1_decode(int bits)
+{
+    int s = (bits >> 3) & 1, e = (bits >> 1) & 3, m = bits & 1;
+    double mag = (e == 0) ? ldexp((double)m, -1)          /* 0.m x 2^(1 - bias) */
+                          : ldexp(1.0 + 0.5 * m, e - 1);  /* 1.m x 2^(e - bias) */
+    return s ? -mag : mag;
+}
+
+static int cmp_double(const void *a, const void *b)
+{
+    double x = *(const double *)a, y = *(const double *)b;
+    return (x > y) - (x < y);
+}
+
+NF4O_EXPORT int nf4o_levels(int type, float L[16])
+{
+    if (type == NF4O_TYPE_NF4) {
+        nf4o_codebook(nf4o_default_delta(), L);
+        return 0;
+    }
+    if (type == NF4O_TYPE_INT4) {
+        for (int i = 0; i < 16; ++i) L[i] = (float)((2.0 * i - 15.0) / 15.0);
+        return 0;
+    }
+    if (type == NF4O_TYPE_FP4) {
+        double v[16];
+        for (int b = 0; b < 16; ++b) v[b] = e2m1_decode(b);
+        qsort(v, 16, sizeof(double), cmp_double);
+        double top = v[15];
+        int n = 0;
+        for (int b = 0; b < 16; ++b)
+            if (n == 0 || v[b] != v[n - 1]) v[n++] = v[b];   /* -0 == +0: one level */
+        for (int i = 0; i < n; ++i)
+            if (v[i] == 0.0) v[i] = 0.0;                      /* the zero level is +0 */
+        for (int i = 0; i < 16; ++i) L[i] = (float)(v[i < n ? i : n - 1] / top);
+        return 0;
+    }
+    return -1;
+}
+
+/* ---------------------------------------------------------------------- */
 /* Storage sizes.                                                         */
 /* ---------------------------------------------------------------------- */
 
+/* With double quantization (bs2 > 0): one E4M3 byte per block, one float c2
+ * per group of bs2 blocks and one float mean.  Without it (bs2 == 0): the
+ * block absmax stored as one fp32 per block (reported in *absmax_q), no c2,
+ * no mean (creativeworksofknowledge, "2. Double quantization": the constants
+ * go FP32 -> FP8). */
 NF4O_EXPORT void nf4o_storage_bytes(int64_t numel, int bs, int bs2,
                                     int64_t *codes, int64_t *absmax_q,
                                     int64_t *absmax_c2, int64_t *mean)
 {
     int64_t nblocks = (numel + bs - 1) / bs;
     *codes = (numel + 1) / 2;
+    if (bs2 == 0) {
+        *absmax_q = 4 * nblocks;                /* one float per block */
+        *absmax_c2 = 0;
+        *mean = 0;
+        return;
+    }
     *absmax_q = nblocks;                       /* one FP8 byte per block */
     *absmax_c2 = 4 * ((nblocks + bs2 - 1) / bs2);   /* one float per group */
     *mean = 4;                                  /* one float per tensor */
@@ -288,6 +363,21 @@ NF4O_EXPORT void nf4o_dequant(const uint8_t *packed, const uint8_t *q,
         uint8_t byte = packed[i / 2];
         int code = (i % 2 == 0) ? (byte >> 4) : (byte & 15);
         float v = L[code] * c1p;
+        out[i] = nf4o_bf16_rne(v);
+    }
+}
+
+/* Dequantization without double quantization: the block's fp32 absmax is
+ * the constant, w' = bf16_RNE(L[code] * c1). */
+NF4O_EXPORT void nf4o_dequant_f32(const uint8_t *packed, const float *c1,
+                                  int64_t numel, int bs, const float L[16],
+                                  uint16_t *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < numel; ++i) {
+        uint8_t byte = packed[i / 2];
+        int code = (i % 2 == 0) ? (byte >> 4) : (byte & 15);
+        float v = L[code] * c1[i / bs];
         out[i] = nf4o_bf16_rne(v);
     }
 }

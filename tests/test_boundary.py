@@ -193,3 +193,60 @@ def test_selftest_rejects_limits_out_of_range():
     assert lib.qlora_selftest_bounded_wait(-1, None, None) == ERR_SHAPE
     assert lib.qlora_selftest_bounded_wait(100000001, None, None) == ERR_SHAPE
     assert lib.qlora_selftest_bounded_wait(1000, ctypes.c_void_p(0x40002), None) == ERR_ALIGN
+
+
+@pytest.mark.parametrize("quant_type", ["nf4", "fp4", "int4"])
+def test_levels_match_oracle_bit_for_bit(quant_type):
+    """The library builds each 4-bit type's table itself; it must equal the
+    oracle's, bit for bit (+0 included)."""
+    ours = np.array(qb.qlora_get_levels(quant_type), dtype=np.float32)
+    assert ours.view(np.uint32).tolist() == oracle.levels(quant_type).view(np.uint32).tolist()
+    out = (ctypes.c_float * 16)()
+    assert lib.qlora_get_levels(3, out) == ERR_UNSUP
+    assert lib.qlora_get_levels(0, None) == ERR_NULL
+
+
+@pytest.mark.parametrize("rows,cols", [(4096, 4096), (3, 100), (22016, 8192), (1, 1)])
+def test_sizes_without_double_quant_match_oracle(rows, cols):
+    sz = qb.qlora_nf4_sizes(rows, cols, double_quant=False)
+    ref = oracle.storage_bytes(rows * cols, 64, 0)
+    assert (sz["codes"], sz["absmax_q"], sz["absmax_c2"]) == (ref["codes"], ref["absmax_q"], ref["absmax_c2"])
+    assert sz["workspace"] >= 8 * 148                  # the encoder's per-CTA partial sums only
+
+
+def test_variant_descriptor_validation():
+    w, ws = ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000)
+    bad_type = _tensor()
+    bad_type.quant_type = 3
+    assert lib.qlora_quantize_nf4_dq(w, ctypes.byref(bad_type), ws, 1 << 40, None) == ERR_UNSUP
+    assert lib.qlora_dequantize(ctypes.byref(bad_type), w, None) == ERR_UNSUP
+    rsv = _tensor()
+    rsv.reserved = 1
+    assert lib.qlora_dequantize(ctypes.byref(rsv), w, None) == ERR_UNSUP
+    plain = _tensor()
+    plain.blocksize2 = 0                        # fp32 constants: `absmax` is required, the rest ignored
+    assert lib.qlora_dequantize(ctypes.byref(plain), w, None) == ERR_NULL
+    plain.absmax = 0x50008
+    assert lib.qlora_dequantize(ctypes.byref(plain), w, None) == ERR_ALIGN
+    plain.absmax = 0x50000
+    plain.absmax_q = plain.absmax_c2 = plain.absmax_mean = None
+    # passes validation; without a GPU it can only fail at the device query
+    assert lib.qlora_dequantize(ctypes.byref(plain), w, None) not in (ERR_NULL, ERR_ALIGN, ERR_UNSUP, ERR_SHAPE)
+    small_ws = lib.qlora_quantize_nf4_dq(w, ctypes.byref(plain), ws, 8 * 2048 - 8, None)
+    assert small_ws == ERR_WS
+
+
+def test_multi_adapter_validation_before_launch():
+    t = _tensor(256, 256)
+    p = ctypes.c_void_p(0x40000)
+    s = ctypes.c_float(2.0)
+    idx = ctypes.c_void_p(0x60000)
+    f = lib.qlora_linear_fwd_multi
+    assert f(ctypes.byref(t), p, 17, p, p, 2, idx, 8, s, p, None, p, 1 << 40, None) == ERR_SHAPE   # M > 16
+    assert f(ctypes.byref(t), p, 4, p, p, 0, idx, 8, s, p, None, p, 1 << 40, None) == ERR_SHAPE    # no adapter
+    assert f(ctypes.byref(t), p, 4, p, p, 2, None, 8, s, p, None, p, 1 << 40, None) == ERR_NULL
+    assert f(ctypes.byref(t), p, 4, p, p, 2, ctypes.c_void_p(0x60002), 8, s, p, None, p, 1 << 40,
+             None) == ERR_ALIGN
+    assert f(ctypes.byref(t), p, 4, p, ctypes.c_void_p(0x40008), 2, idx, 8, s, p, None, p, 1 << 40,
+             None) == ERR_ALIGN
+    assert f(ctypes.byref(t), p, 4, p, p, 2, idx, 8, s, p, None, p, 16, None) == ERR_WS

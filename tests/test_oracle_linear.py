@@ -103,3 +103,37 @@ def test_gradients_are_lora_only_and_scale_linearly():
     dX2, dA2, dB2 = oracle.linear_bwd(Wd, X, dY, A, B, 2.0)
     assert np.allclose(dA2, 2 * dA1, rtol=1e-13, atol=0) and np.allclose(dB2, 2 * dB1, rtol=1e-13, atol=0)
     assert dA1.shape == A.shape and dB1.shape == B.shape and dX1.shape == X.shape
+
+
+def test_multi_adapter_forward_properties():
+    """Per-token adapters: one adapter for every token reduces to the single-
+    adapter forward; a negative index means the base weight alone; permuting
+    the tokens together with their indices permutes the rows; an adapter no
+    token uses changes nothing; zero B_a removes exactly adapter a's term."""
+    Wd, X, A, B, dY = _case(m=12, n=40, k=128, r=8, proj=5)
+    rng = np.random.Generator(np.random.PCG64(7))
+    A_st = np.stack([A, 0.5 * A[::-1], rng.standard_normal(A.shape).astype(np.float32) * 0.02])
+    B_st = np.stack([B, -B, rng.standard_normal(B.shape).astype(np.float32) * 0.02])
+    s = 2.0
+    for a in range(3):
+        Y1, XA1 = oracle.linear_fwd_multi(Wd, X, A_st, B_st, np.full(12, a), s)
+        Y2, XA2 = oracle.linear_fwd(Wd, X, A_st[a], B_st[a], s)
+        assert np.max(np.abs(Y1 - Y2)) <= 1e-12 * np.sqrt(np.mean(Y2 ** 2))
+        assert np.max(np.abs(XA1 - XA2)) <= 1e-12 * np.sqrt(np.mean(XA2 ** 2))
+    base = X.astype(np.float64) @ Wd.T.astype(np.float64)
+    Yn, XAn = oracle.linear_fwd_multi(Wd, X, A_st, B_st, np.full(12, -1), s)
+    assert np.array_equal(Yn, base) and np.all(XAn == 0)
+    idx = np.array([0, 1, 2, -1, 2, 2, 0, 1, 1, 0, 2, 1])
+    Y, XA = oracle.linear_fwd_multi(Wd, X, A_st, B_st, idx, s)
+    perm = rng.permutation(12)
+    Yp, XAp = oracle.linear_fwd_multi(Wd, X[perm], A_st, B_st, idx[perm], s)
+    assert np.max(np.abs(Yp - Y[perm])) < 1e-12 and np.max(np.abs(XAp - XA[perm])) < 1e-12
+    A4 = np.concatenate([A_st, A_st[:1] * 3])
+    B4 = np.concatenate([B_st, B_st[:1] * 3])
+    Y4, _ = oracle.linear_fwd_multi(Wd, X, A4, B4, idx, s)
+    assert np.max(np.abs(Y4 - Y)) < 1e-12
+    Bz = B_st.copy()
+    Bz[1] = 0
+    Yz, _ = oracle.linear_fwd_multi(Wd, X, A_st, Bz, idx, s)
+    assert np.max(np.abs(Yz[idx == 1] - base[idx == 1])) < 1e-12
+    assert np.max(np.abs(Yz[idx != 1] - Y[idx != 1])) < 1e-12
