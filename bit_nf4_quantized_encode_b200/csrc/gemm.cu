@@ -454,8 +454,8 @@ cudaError_t launch_fused_t(const FusedArgs& args, const CUtensorMap& act, const 
 cudaError_t launch_fused(FusedDir dir, int token_tile, const FusedArgs& args, const CUtensorMap& act,
                          const CUtensorMap& lora_act, int num_sms, cudaStream_t stream) {
   if (dir == FusedDir::kFwd) {
+    // the decode-shaped forward (16 tokens or fewer) is k_gemv's
     if (token_tile == 256) return launch_fused_t<0, 256>(args, act, lora_act, num_sms, stream);
-    if (token_tile == 16) return launch_fused_t<0, 16>(args, act, lora_act, num_sms, stream);
   } else {
     if (token_tile == 256) return launch_fused_t<1, 256>(args, act, lora_act, num_sms, stream);
     if (token_tile == 16) return launch_fused_t<1, 16>(args, act, lora_act, num_sms, stream);

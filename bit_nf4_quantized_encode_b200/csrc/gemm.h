@@ -44,8 +44,8 @@ struct FusedArgs {
   uint32_t* err;             // device error flag
 };
 
-// Token tile of the fused kernel: 256 for prefill-shaped calls, 16 for
-// decode-shaped calls (M <= 16).
+// Token tile of the fused kernel: 256 for prefill-shaped calls; the backward
+// also takes 16 for decode-shaped calls (M <= 16).
 cudaError_t launch_fused(FusedDir dir, int token_tile, const FusedArgs& args, const CUtensorMap& act,
                          const CUtensorMap& lora_act, int num_sms, cudaStream_t stream);
 // out[i * ld_out + j] = bf16(scale * in[i * ld_in + j]) for j < cols_in, 0 for
