@@ -73,6 +73,9 @@ __global__ void __launch_bounds__(256) k_encode(const uint16_t* __restrict__ w, 
     s_base[i] = tab.bucket_base[i];
   }
   __syncthreads();
+  // launched as a programmatic dependent: the previous kernel in the stream may
+  // still be running; nothing in global memory is read or written before it ends
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const uint32_t fast_tbl = static_cast<uint32_t>(__cvta_generic_to_shared(s_fast));
   const bool fast_ok = tab.fast != 0;
 
@@ -204,6 +207,7 @@ __global__ void __launch_bounds__(256) k_double_quant(const float* __restrict__ 
                                                       float* __restrict__ c2, float* __restrict__ mean_out) {
   __shared__ double s_red[256];
   asm volatile("griddepcontrol.wait;" ::: "memory");   // k_encode complete
+  asm volatile("griddepcontrol.launch_dependents;");   // a dependent waits for this grid itself
   double t = 0.0;
   for (int i = threadIdx.x; i < npartials; i += blockDim.x) t += partials[i];
   s_red[threadIdx.x] = t;
@@ -283,6 +287,10 @@ __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ cod
                                                  const float* __restrict__ absf, int64_t numel,
                                                  CodebookParam cb, uint16_t* __restrict__ out) {
   __shared__ __align__(16) uint8_t s_out[8][32 * 80];
+  // a programmatic dependent of the previous kernel in the stream: wait for it
+  // before touching global memory, then let the next one launch
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
   const bool plain = absf != nullptr;                // fp32 block constants, no double quantization
   const float mu = plain ? 0.0f : __ldg(mean);
   const int64_t nfull = numel / 32;                  // chunks of 32 real weights
@@ -345,16 +353,11 @@ __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ cod
 }
 
 // ------------------------------------------------------------------ launchers
-cudaError_t launch_encode(const uint16_t* w, int64_t numel, const EncodeTables& tab, uint8_t* codes,
-                          float* c1buf, double* partials, int grid, cudaStream_t stream) {
-  k_encode<<<grid, 256, 0, stream>>>(w, numel, tab, codes, c1buf, partials);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_double_quant(const float* c1buf, int64_t nblocks, const double* partials,
-                                int npartials, uint8_t* q, float* c2, float* mean, int grid,
-                                cudaStream_t stream) {
-  // programmatic dependent of k_encode: the launch overlaps the encoder's tail
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel in the stream finishes (it waits for that kernel
+// with griddepcontrol.wait before using global memory).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, cudaStream_t stream, Args... args) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(256);
@@ -364,7 +367,19 @@ cudaError_t launch_double_quant(const float* c1buf, int64_t nblocks, const doubl
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_double_quant, c1buf, nblocks, partials, npartials, q, c2, mean);
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+cudaError_t launch_encode(const uint16_t* w, int64_t numel, const EncodeTables& tab, uint8_t* codes,
+                          float* c1buf, double* partials, int grid, cudaStream_t stream) {
+  return launch_pdl(k_encode, grid, stream, w, numel, tab, codes, c1buf, partials);
+}
+
+cudaError_t launch_double_quant(const float* c1buf, int64_t nblocks, const double* partials,
+                                int npartials, uint8_t* q, float* c2, float* mean, int grid,
+                                cudaStream_t stream) {
+  // programmatic dependent of k_encode: the launch overlaps the encoder's tail
+  return launch_pdl(k_double_quant, grid, stream, c1buf, nblocks, partials, npartials, q, c2, mean);
 }
 
 int dequant_ctas_per_sm() {
@@ -382,8 +397,7 @@ int encode_ctas_per_sm() {
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* qabs, const float* c2,
                            const float* mean, const float* absf, int64_t numel, const CodebookParam& cb,
                            uint16_t* out, int grid, cudaStream_t stream) {
-  k_dequant<<<grid, 256, 0, stream>>>(codes, qabs, c2, mean, absf, numel, cb, out);
-  return cudaGetLastError();
+  return launch_pdl(k_dequant, grid, stream, codes, qabs, c2, mean, absf, numel, cb, out);
 }
 
 }  // namespace qlora

@@ -21,6 +21,9 @@ struct CodebookParam {
   float level[16];
 };
 
+// The codec kernels are launched as programmatic dependents of the kernel
+// before them in the stream (each waits for it before touching global memory),
+// so back-to-back calls overlap one launch's start with the previous one's end.
 cudaError_t launch_encode(const uint16_t* w, int64_t numel, const EncodeTables& tab, uint8_t* codes,
                           float* c1buf, double* partials, int grid, cudaStream_t stream);
 // Resident k_encode / k_dequant CTAs per SM (their grids are one wave of them).
