@@ -27,7 +27,7 @@
  * before the second quantization, a codebook with an exact zero: these come
  * from the benchmark spec of this hot path, not from the pages.
  *
- * Readings where the pages are silent (each is listed in the design notes):
+ * Readings where the pages are silent:
  *   R1  codebook: 8 positive quantiles Phi^-1(1/2 + (delta-1/2) j/8), j=1..8,
  *       7 negative ones -Phi^-1(1/2 + (delta-1/2) j/7), j=1..7, plus 0, each
  *       side divided by Phi^-1(delta); delta = 1 - (1/30 + 1/32)/2.
