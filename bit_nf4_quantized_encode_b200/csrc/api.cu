@@ -181,8 +181,8 @@ qlora_status check_linear(const qlora_nf4_tensor* W, int64_t M, int32_t r, Linea
 
 // Work buffer layout: fp32 accumulators first (one memset clears them all),
 // then bf16 staging.  Offsets in bytes, each 256-aligned.
-// Splits of the rank-r contractions are sized for up to this many SMs, so a
-// work buffer sized without a device fits any device's launch.
+// The work buffer's split slots are sized independently of the device (for up
+// to this many SMs); a launch picks its own split count within that space.
 constexpr int kSizingSms = 256;
 constexpr int kMaxRankSplits = 32;
 
@@ -191,22 +191,46 @@ struct RankPlan {
   int m_tiles, n_tiles, ksteps, splits;
   int tiles() const { return m_tiles * n_tiles; }
 };
-RankPlan rank_plan(int64_t mdim, int64_t contraction, int lora_steps, int sms_tiles_total, int num_sms) {
+RankPlan rank_tiling(int64_t mdim, int64_t contraction, int lora_steps) {
   RankPlan p;
   p.m_tiles = static_cast<int>((mdim + 127) / 128);
   p.n_tiles = lora_steps;
   p.ksteps = static_cast<int>((contraction + 63) / 64);
-  p.splits = rank_splits(sms_tiles_total, p.ksteps, num_sms, kMaxRankSplits);
+  p.splits = 1;
   return p;
+}
+// Splits of a launch with `tiles` tiles in all (the problems of one launch
+// share them) and `ksteps` k-steps, within `slot_bytes` of slot space.
+int launch_splits(int tiles, int ksteps, int num_sms, size_t slot_bytes) {
+  // a split count s > 1 needs tiles * s partial tiles of slot space
+  const size_t per_split = static_cast<size_t>(tiles) * 64 * 128 * sizeof(float);
+  size_t cap = kMaxRankSplits;
+  if (per_split > 0 && slot_bytes / per_split < cap) cap = slot_bytes / per_split;
+  return rank_splits(tiles, ksteps, num_sms, cap < 2 ? 1 : static_cast<int>(cap));
+}
+// The plan of a launch must fit its slot region; checked before every launch.
+bool slots_fit(int tiles, int splits, size_t slot_bytes) {
+  return rank_slot_bytes(tiles, splits) <= slot_bytes;
+}
+// Slot space of a launch: the most any of these SM counts plans for, so a
+// buffer sized without a device lets the launch use its own best split count.
+size_t sized_slots(int tiles, int ksteps) {
+  static const int kSmCounts[] = {96, 108, 114, 120, 128, 132, 144, 148, 152, 160, 170, 188, 192, 224, kSizingSms};
+  size_t most = 0;
+  for (int sms : kSmCounts) {
+    const size_t b = rank_slot_bytes(tiles, rank_splits(tiles, ksteps, sms, kMaxRankSplits));
+    if (b > most) most = b;
+  }
+  return most;
 }
 
 // Work buffer layout: the region cleared by one memset first (counters, and
 // the decode backward's split-K dX accumulator), then the rest.  Offsets in
-// bytes, each 256-aligned.
+// bytes, each 256-aligned; every size is independent of the device.
 struct FwdLayout {
-  size_t cnt, slots, xa_slices, sxa, rank_cnt, rank_slots, clear_end, total;
+  size_t cnt, slots, xa_slices, sxa, rank_cnt, rank_slots, rank_slot_bytes, clear_end, total;
 };
-FwdLayout fwd_layout(const LinearShape& s, int num_sms = kSizingSms) {
+FwdLayout fwd_layout(const LinearShape& s) {
   FwdLayout l{};
   size_t o = 0;
   if (s.decode) {        // k_xa_zero + k_gemv: tile counters, partial slots, X A^T slices
@@ -220,11 +244,11 @@ FwdLayout fwd_layout(const LinearShape& s, int num_sms = kSizingSms) {
     return l;
   }
   // k_rank (X A^T -> bf16(s X A^T)) then the fused dequant-GEMM
-  const RankPlan xa = rank_plan(s.m, s.cols, s.lora_steps,
-                                int((s.m + 127) / 128) * s.lora_steps, num_sms);
+  const RankPlan xa = rank_tiling(s.m, s.cols, s.lora_steps);
   l.rank_cnt = o;   o = round_up(o + size_t(xa.tiles()) * 4, 256);
   l.clear_end = o;
-  l.rank_slots = o; o = round_up(o + rank_slot_bytes(xa.tiles(), xa.splits), 256);
+  l.rank_slot_bytes = sized_slots(xa.tiles(), xa.ksteps);
+  l.rank_slots = o; o = round_up(o + l.rank_slot_bytes, 256);
   l.sxa = o;        o = round_up(o + size_t(s.m) * s.rpad * 2, 256);
   l.total = o;
   return l;
@@ -232,30 +256,30 @@ FwdLayout fwd_layout(const LinearShape& s, int num_sms = kSizingSms) {
 
 // Backward: launch 1 = dY B (and X A^T when it is not supplied), launch 2 =
 // the fused dX, launch 3 = dY^T (s X A^T) and X^T (s dY B) (more than 16
-// tokens; with fewer, k_small_grads from the fp32 G and X A^T).
+// tokens; with fewer, k_small_grads from the fp32 G and X A^T).  Launch 1's
+// slot space covers both of its forms.
 struct BwdLayout {
-  size_t cnt1, cnt2, dx_acc, clear_end, slots1, slots2, g, xa, sg, sxa, total;
+  size_t cnt1, cnt2, dx_acc, clear_end, slots1, slots1_bytes, slots2, slots2_bytes, g, xa, sg, sxa, total;
   RankPlan g_plan, xa_plan, db_plan, da_plan;
 };
-BwdLayout bwd_layout(const LinearShape& s, int num_sms = kSizingSms) {
+BwdLayout bwd_layout(const LinearShape& s) {
   BwdLayout l{};
-  // launch 1 is planned for both problems whether or not X A^T is recomputed,
-  // so that the layout does not depend on the call
-  const int t1 = 2 * int((s.m + 127) / 128) * s.lora_steps;
-  l.g_plan = rank_plan(s.m, s.rows, s.lora_steps, t1, num_sms);
-  l.xa_plan = rank_plan(s.m, s.cols, s.lora_steps, t1, num_sms);
-  const int t2 = int((s.rows + 127) / 128 + (s.cols + 127) / 128) * s.lora_steps;
-  l.db_plan = rank_plan(s.rows, s.m, s.lora_steps, t2, num_sms);
-  l.da_plan = rank_plan(s.cols, s.m, s.lora_steps, t2, num_sms);
+  l.g_plan = rank_tiling(s.m, s.rows, s.lora_steps);
+  l.xa_plan = rank_tiling(s.m, s.cols, s.lora_steps);
+  l.db_plan = rank_tiling(s.rows, s.m, s.lora_steps);
+  l.da_plan = rank_tiling(s.cols, s.m, s.lora_steps);
+  const int k1 = l.g_plan.ksteps > l.xa_plan.ksteps ? l.g_plan.ksteps : l.xa_plan.ksteps;
+  const size_t alone = sized_slots(l.g_plan.tiles(), l.g_plan.ksteps);
+  const size_t both = sized_slots(l.g_plan.tiles() + l.xa_plan.tiles(), k1);
+  l.slots1_bytes = alone > both ? alone : both;
+  l.slots2_bytes = s.decode ? 0 : sized_slots(l.db_plan.tiles() + l.da_plan.tiles(), l.db_plan.ksteps);
   size_t o = 0;
   l.cnt1 = o;   o = round_up(o + size_t(l.g_plan.tiles() + l.xa_plan.tiles()) * 4, 256);
   l.cnt2 = o;   o = round_up(o + size_t(l.db_plan.tiles() + l.da_plan.tiles()) * 4, 256);
   l.dx_acc = o; if (s.decode) o = round_up(o + size_t(s.m) * s.cols * 4, 256);
   l.clear_end = o;
-  l.slots1 = o; o = round_up(o + rank_slot_bytes(l.g_plan.tiles(), l.g_plan.splits) +
-                             rank_slot_bytes(l.xa_plan.tiles(), l.xa_plan.splits), 256);
-  l.slots2 = o; if (!s.decode) o = round_up(o + rank_slot_bytes(l.db_plan.tiles(), l.db_plan.splits) +
-                                            rank_slot_bytes(l.da_plan.tiles(), l.da_plan.splits), 256);
+  l.slots1 = o; o = round_up(o + l.slots1_bytes, 256);
+  l.slots2 = o; o = round_up(o + l.slots2_bytes, 256);
   l.g = o;      if (s.decode) o = round_up(o + size_t(s.m) * s.rpad * 4, 256);
   l.xa = o;     if (s.decode) o = round_up(o + size_t(s.m) * s.rpad * 4, 256);
   l.sg = o;     o = round_up(o + size_t(s.m) * s.rpad * 2, 256);
@@ -516,12 +540,10 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor* W, const uint16_t* X, int6
       (XA_out && !aligned16(XA_out)))
     return QLORA_ERR_ALIGN;
   if (!std::isfinite(s)) return QLORA_ERR_SHAPE;
-  // the size check uses the device-independent layout (an upper bound of the
-  // one the launch uses, which depends on the SM count)
-  if (workspace_bytes < fwd_layout(sh).total) return QLORA_ERR_WORKSPACE;
+  const FwdLayout L = fwd_layout(sh);
+  if (workspace_bytes < L.total) return QLORA_ERR_WORKSPACE;
   DeviceInfo d;
   if ((st = device_info(&d)) != QLORA_OK) return st;
-  const FwdLayout L = fwd_layout(sh, d.num_sms);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
 
@@ -531,7 +553,9 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor* W, const uint16_t* X, int6
   // 1) X A^T (fp32 to XA_out when asked) and bf16(s X A^T), zero-padded to a
   //    multiple of 64 columns, as the LoRA k-step operand of the fused GEMM
   uint16_t* sxa = reinterpret_cast<uint16_t*>(ws + L.sxa);
-  const RankPlan xp = rank_plan(sh.m, sh.cols, sh.lora_steps, int((sh.m + 127) / 128) * sh.lora_steps, d.num_sms);
+  RankPlan xp = rank_tiling(sh.m, sh.cols, sh.lora_steps);
+  xp.splits = launch_splits(xp.tiles(), xp.ksteps, d.num_sms, L.rank_slot_bytes);
+  if (!slots_fit(xp.tiles(), xp.splits, L.rank_slot_bytes)) return QLORA_ERR_WORKSPACE;
   if (xp.splits > 1 && cudaMemsetAsync(ws, 0, L.clear_end, cs) != cudaSuccess) return QLORA_ERR_CUDA;
   CUtensorMap x_k, a_k;
   if (!make_map(&x_k, X, sh.cols, sh.m, sh.cols * 2, 128) ||
@@ -586,12 +610,10 @@ qlora_status qlora_linear_fwd_multi(const qlora_nf4_tensor* W, const uint16_t* X
       (XA_out && !aligned16(XA_out)) || (reinterpret_cast<uintptr_t>(adapter_idx) & 3u) != 0)
     return QLORA_ERR_ALIGN;
   if (!std::isfinite(s)) return QLORA_ERR_SHAPE;
-  // the size check uses the device-independent layout (an upper bound of the
-  // one the launch uses, which depends on the SM count)
-  if (workspace_bytes < fwd_layout(sh).total) return QLORA_ERR_WORKSPACE;
+  const FwdLayout L = fwd_layout(sh);
+  if (workspace_bytes < L.total) return QLORA_ERR_WORKSPACE;
   DeviceInfo d;
   if ((st = device_info(&d)) != QLORA_OK) return st;
-  const FwdLayout L = fwd_layout(sh, d.num_sms);
   return run_decode_fwd(W, X, sh, A_stack, B_stack, adapter_idx, n_adapters, s, Y, XA_out,
                         static_cast<uint8_t*>(workspace), L, d, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -608,10 +630,10 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor* W, const uint16_t* X, cons
       !aligned16(dB) || !aligned16(workspace) || (XA && !aligned16(XA)) || (dX && !aligned16(dX)))
     return QLORA_ERR_ALIGN;
   if (!std::isfinite(s)) return QLORA_ERR_SHAPE;
-  if (workspace_bytes < bwd_layout(sh).total) return QLORA_ERR_WORKSPACE;
+  BwdLayout L = bwd_layout(sh);
+  if (workspace_bytes < L.total) return QLORA_ERR_WORKSPACE;
   DeviceInfo d;
   if ((st = device_info(&d)) != QLORA_OK) return st;
-  const BwdLayout L = bwd_layout(sh, d.num_sms);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* dx_acc = reinterpret_cast<float*>(ws + L.dx_acc);
@@ -632,6 +654,16 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor* W, const uint16_t* X, cons
       !make_map(&a_k, A, sh.cols, sh.r, sh.cols * 2, 64))
     return QLORA_ERR_CUDA;
   {
+    // splits for this device and this form of launch 1, within the slot space
+    if (recompute) {
+      const int k1 = L.g_plan.ksteps > L.xa_plan.ksteps ? L.g_plan.ksteps : L.xa_plan.ksteps;
+      L.g_plan.splits = L.xa_plan.splits =
+          launch_splits(L.g_plan.tiles() + L.xa_plan.tiles(), k1, d.num_sms, L.slots1_bytes);
+    } else {
+      L.g_plan.splits = launch_splits(L.g_plan.tiles(), L.g_plan.ksteps, d.num_sms, L.slots1_bytes);
+    }
+    if (!slots_fit(L.g_plan.tiles() + (recompute ? L.xa_plan.tiles() : 0), L.g_plan.splits, L.slots1_bytes))
+      return QLORA_ERR_WORKSPACE;
     RankArgs ra{};
     uint32_t* cnt = reinterpret_cast<uint32_t*>(ws + L.cnt1);
     float* slots = reinterpret_cast<float*>(ws + L.slots1);
@@ -703,6 +735,10 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor* W, const uint16_t* X, cons
       !make_map(&x_mn, X, sh.cols, sh.m, sh.cols * 2, 64) ||
       !make_map(&sg_mn, sg, sh.rpad, sh.m, sh.rpad * 2, 64))
     return QLORA_ERR_CUDA;
+  L.db_plan.splits = L.da_plan.splits =
+      launch_splits(L.db_plan.tiles() + L.da_plan.tiles(), L.db_plan.ksteps, d.num_sms, L.slots2_bytes);
+  if (!slots_fit(L.db_plan.tiles() + L.da_plan.tiles(), L.db_plan.splits, L.slots2_bytes))
+    return QLORA_ERR_WORKSPACE;
   RankArgs rb{};
   uint32_t* cnt2 = reinterpret_cast<uint32_t*>(ws + L.cnt2);
   float* slots2 = reinterpret_cast<float*>(ws + L.slots2);

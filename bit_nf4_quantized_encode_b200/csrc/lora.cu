@@ -162,21 +162,31 @@ k_rank(const RankArgs a, const __grid_constant__ CUtensorMap am0, const __grid_c
         const RankProblem& p = a.p[w.prob];
         const CUtensorMap* am = w.prob ? &am1 : &am0;
         const CUtensorMap* bm = w.prob ? &bm1 : &bm0;
-        for (int j = 0; j < w.nk; ++j, ++it) {
-          const uint32_t stage = it % kStages, phase = (it / kStages) & 1u;
-          if (!mbar_wait(&empty[stage], phase ^ 1u, a.err)) { alive = false; break; }
-          uint8_t* sA = smem_gen + stage * kStageBytes;
-          uint8_t* sB = sA + kABytes;
-          const int k0 = (w.kbeg + j) * 64;
-          mbar_arrive_expect_tx(&full[stage], kStageBytes);
-          if (p.a_mn) {   // A^T stored [k][m]: two 64-wide MN boxes
-            tma_load_2d(sA, am, w.mt * 128, k0, &full[stage]);
-            tma_load_2d(sA + 8192, am, w.mt * 128 + 64, k0, &full[stage]);
-          } else {
-            tma_load_2d(sA, am, k0, w.mt * 128, &full[stage]);
+        // two consecutive k-steps at a time: both stages are claimed first and
+        // their loads issued back to back, so every row of the long operand is
+        // requested in 256-byte runs rather than 128-byte ones
+        for (int j = 0; j < w.nk && alive; j += 2) {
+          const int cnt = w.nk - j < 2 ? w.nk - j : 2;
+          for (int q = 0; q < cnt; ++q) {
+            const uint32_t stage = (it + q) % kStages, phase = ((it + q) / kStages) & 1u;
+            if (!mbar_wait(&empty[stage], phase ^ 1u, a.err)) { alive = false; break; }
           }
-          if (p.b_mn) tma_load_2d(sB, bm, w.nt * 64, k0, &full[stage]);
-          else tma_load_2d(sB, bm, k0, w.nt * 64, &full[stage]);
+          if (!alive) break;
+          for (int q = 0; q < cnt; ++q, ++it) {
+            const uint32_t stage = it % kStages;
+            uint8_t* sA = smem_gen + stage * kStageBytes;
+            uint8_t* sB = sA + kABytes;
+            const int k0 = (w.kbeg + j + q) * 64;
+            mbar_arrive_expect_tx(&full[stage], kStageBytes);
+            if (p.a_mn) {   // A^T stored [k][m]: two 64-wide MN boxes
+              tma_load_2d(sA, am, w.mt * 128, k0, &full[stage]);
+              tma_load_2d(sA + 8192, am, w.mt * 128 + 64, k0, &full[stage]);
+            } else {
+              tma_load_2d(sA, am, k0, w.mt * 128, &full[stage]);
+            }
+            if (p.b_mn) tma_load_2d(sB, bm, w.nt * 64, k0, &full[stage]);
+            else tma_load_2d(sB, bm, k0, w.nt * 64, &full[stage]);
+          }
         }
       }
     }
@@ -316,11 +326,26 @@ std::atomic<uint64_t> g_attr_done{0};
 }  // namespace
 
 int rank_splits(int tiles, int ksteps, int num_sms, int max_splits) {
-  int s = tiles > 0 ? num_sms / tiles : 1;
+  // makespan model: waves of units over the SMs times the k-steps of a unit
+  // plus two k-steps of fixed cost (epilogue, split fix-up)
+  // each split adds a 32 KB partial tile written and read back: beyond the
+  // splits a tile needs to spread over the SMs (about two units per SM), at
+  // most 4
+  int spread = tiles > 0 ? (2 * num_sms + tiles - 1) / tiles : 1;
+  if (spread < 4) spread = 4;
+  if (max_splits > spread) max_splits = spread;
+  int best = 1;
+  int64_t best_cost = -1;
   const int cap = ksteps / 4 > 1 ? ksteps / 4 : 1;          // at least 4 k-steps per split
-  if (s > cap) s = cap;
-  if (s > max_splits) s = max_splits;
-  return s < 1 ? 1 : s;
+  for (int s = 1; s <= max_splits && s <= cap; ++s) {
+    const int64_t waves = (static_cast<int64_t>(tiles) * s + num_sms - 1) / num_sms;
+    const int64_t cost = waves * ((ksteps + s - 1) / s + 2);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
 }
 
 size_t rank_slot_bytes(int tiles, int splits) {

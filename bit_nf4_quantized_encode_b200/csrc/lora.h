@@ -47,8 +47,10 @@ struct RankArgs {
   uint32_t* err;
 };
 
-// K splits for `tiles` output tiles of `ksteps` k-steps: enough units to fill
-// the SMs, at least 4 k-steps per split, at most max_splits.
+// K splits for `tiles` output tiles of `ksteps` k-steps: the count that
+// minimises waves-of-units x k-steps-per-unit over num_sms SMs, with at least
+// 4 k-steps per split and at most max(4, ceil(2 num_sms / tiles)) and
+// max_splits splits.
 int rank_splits(int tiles, int ksteps, int num_sms, int max_splits);
 // Bytes of the partial-tile slots of a problem.
 size_t rank_slot_bytes(int tiles, int splits);
