@@ -787,23 +787,35 @@ k_xa_zero(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A, int64_
   }
   for (int64_t ch = c_beg + threadIdx.x; ch < c_end; ch += blockDim.x) {
     float af[4][8];
-    if constexpr (!kMulti) load_a_rows(A, j0, r, kw, ch, af);   // shared by every token
-    uint4 xv[kMaxM];
+    if constexpr (!kMulti) {
+      load_a_rows(A, j0, r, kw, ch, af);     // shared by every token
+      uint4 xv[kMaxM];
 #pragma unroll
-    for (int i = 0; i < kMaxM; ++i)
-      xv[i] = i < mi ? __ldg(reinterpret_cast<const uint4*>(X + i * kw) + ch) : make_uint4(0u, 0u, 0u, 0u);
+      for (int i = 0; i < kMaxM; ++i)
+        xv[i] = i < mi ? __ldg(reinterpret_cast<const uint4*>(X + i * kw) + ch) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-    for (int i = 0; i < kMaxM; ++i) {
-      if constexpr (kMulti) {
+      for (int i = 0; i < kMaxM; ++i) {
+        const float xf[8] = {bf16_lo(xv[i].x), bf16_hi(xv[i].x), bf16_lo(xv[i].y), bf16_hi(xv[i].y),
+                             bf16_lo(xv[i].z), bf16_hi(xv[i].z), bf16_lo(xv[i].w), bf16_hi(xv[i].w)};
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[c][i] = __fmaf_rn(af[c][e], xf[e], acc[c][i]);
+      }
+    } else {
+      // one token at a time: its own adapter's A rows and its X chunk
+#pragma unroll
+      for (int i = 0; i < kMaxM; ++i) {
         if (ad[i] < 0) continue;
         load_a_rows(A + static_cast<int64_t>(ad[i]) * a_stride, j0, r, kw, ch, af);
+        const uint4 xv = __ldg(reinterpret_cast<const uint4*>(X + i * kw) + ch);
+        const float xf[8] = {bf16_lo(xv.x), bf16_hi(xv.x), bf16_lo(xv.y), bf16_hi(xv.y),
+                             bf16_lo(xv.z), bf16_hi(xv.z), bf16_lo(xv.w), bf16_hi(xv.w)};
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[c][i] = __fmaf_rn(af[c][e], xf[e], acc[c][i]);
       }
-      const float xf[8] = {bf16_lo(xv[i].x), bf16_hi(xv[i].x), bf16_lo(xv[i].y), bf16_hi(xv[i].y),
-                           bf16_lo(xv[i].z), bf16_hi(xv[i].z), bf16_lo(xv[i].w), bf16_hi(xv[i].w)};
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[c][i] = __fmaf_rn(af[c][e], xf[e], acc[c][i]);
     }
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

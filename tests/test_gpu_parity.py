@@ -281,3 +281,30 @@ def test_linear_gemv_65b_ffn(qb, n, k, m):
     """The decode-shaped forward on the 65B FFN weights (22016 x 8192 and
     8192 x 22016) at 1, 4 and 16 tokens, r = 64: every output compared."""
     _linear_case(qb, n, k, m, 64, 16.0, proj=5 if n > k else 6, check_bwd=False)
+
+
+@pytest.mark.parametrize("n,k,m", [(22016, 8192, 1024), (392, 640, 300), (4096, 4096, 16)])
+def test_results_are_bit_reproducible(qb, n, k, m):
+    """The split contractions sum their partial tiles in a fixed order, so two
+    identical calls give the same bits (outputs poisoned in between):
+    Y, X A^T, dA, dB always, and dX with more than 16 tokens."""
+    qt, _ = _oracle_weight(n, k, 2)
+    up = _upload_oracle_quant(qb, qt)
+    X, A = workloads.activations(m, k, 2).cuda(), workloads.lora_a(64, k, 2).cuda()
+    B, dY = workloads.lora_b(n, 64, 2).cuda(), workloads.grad_output(m, n, 2).cuda()
+    runs = []
+    for _ in range(2):
+        Y = torch.full((m, n), float("nan"), dtype=torch.bfloat16, device="cuda")
+        XA = torch.full((m, 64), float("nan"), dtype=torch.float32, device="cuda")
+        qb.qlora_linear_fwd(up, X, A, B, 0.25, Y=Y, XA=XA)
+        dX, dA, dB = qb.qlora_linear_bwd(up, X, dY, A, B, 0.25, XA=XA)
+        xa_again = qb.qlora_linear_bwd(up, X, dY, A, B, 0.25, XA=None, need_dx=False)  # X A^T recomputed
+        torch.cuda.synchronize()
+        runs.append([t.cpu().view(torch.int16 if t.dtype == torch.bfloat16 else torch.int32)
+                     for t in (Y, XA, dA, dB, dX, xa_again[1], xa_again[2])])
+    assert qb.qlora_read_device_errors() == 0
+    names = ["Y", "XA", "dA", "dB", "dX", "dA (X A^T recomputed)", "dB (X A^T recomputed)"]
+    for name, a, b in zip(names, runs[0], runs[1]):
+        if name == "dX" and m <= 16:
+            continue                                  # split-K fp32 atomics at 16 tokens or fewer
+        assert torch.equal(a, b), f"{name} differs between two identical calls ({n}x{k}, m={m})"
