@@ -55,10 +55,24 @@ __device__ __forceinline__ void lookup4(uint32_t w16, const ByteTables& t, uint3
   out23 = __byte_perm(l, h, 0x6273);   // element 2 (nibble 3), element 3 (nibble 2)
 }
 
+// The two byte-permute stages of lookup4 given their selectors: s holds the
+// low 3 bits of each code (table half index), s2 picks the half by code bit 3.
+__device__ __forceinline__ void lookup4_sel(uint32_t s, uint32_t s2, const ByteTables& t, uint32_t& out01,
+                                            uint32_t& out23) {
+  const uint32_t h = __byte_perm(__byte_perm(t.ha0, t.ha1, s), __byte_perm(t.hb0, t.hb1, s), s2);
+  const uint32_t l = __byte_perm(__byte_perm(t.la0, t.la1, s), __byte_perm(t.lb0, t.lb1, s), s2);
+  out01 = __byte_perm(l, h, 0x4051);
+  out23 = __byte_perm(l, h, 0x6273);
+}
+
+// Eight codes -> four bf16x2 words: the selectors of all eight codes are
+// built at once (byte-permute reads only the low 16 bits of a selector).
 __device__ __forceinline__ uint4 expand8(uint32_t w, const ByteTables& t) {
+  const uint32_t s = w & 0x77777777u;
+  const uint32_t s2 = ((w >> 1) & 0x44444444u) | 0x32103210u;
   uint4 o;
-  lookup4(w & 0xFFFFu, t, o.x, o.y);
-  lookup4(w >> 16, t, o.z, o.w);
+  lookup4_sel(s, s2, t, o.x, o.y);
+  lookup4_sel(s >> 16, s2 >> 16, t, o.z, o.w);
   return o;
 }
 
