@@ -24,10 +24,15 @@
 //     warp MMAs (m16n8k16, bf16 in, fp32 out): a code byte is exactly one
 //     A-fragment register.  The block's product is scaled by its constant and
 //     added to fp32 registers.
-//   * Each warp writes its fp32 partial of a tile to one of its CTA's two
-//     slots; the warp whose partial completes a tile's 32 rows (a per-warp
-//     counter) sums the slots of the tile's CTAs, adds the LoRA up-projection
-//     with warp MMAs over the staged bf16(s X A^T) and writes those rows of Y.
+//   * A tile that lies in one CTA's share is finished by that CTA at once.
+//     For a shared tile each warp writes its fp32 partial to one of its CTA's
+//     two slots; the warp whose partial completes the tile's 32 rows (a
+//     per-warp counter) sums the slots of the tile's CTAs, adds the LoRA
+//     up-projection with warp MMAs over the staged bf16(s X A^T) and writes
+//     those rows of Y.  At the end of its share a warp that finds every other
+//     part already counted finishes without writing or counting its own.
+//   * The producer warpgroup gives registers to the consumers after the start
+//     (setmaxnreg), so that the consumers' loop runs without spills.
 //   * The tensor core here only replaces FMAs: per weight it does 2 M FLOP.
 //     Warp MMAs are used because a skinny-N product issued as tcgen05.mma
 //     from one thread costs about 80 cycles per 128x16x16 instruction, which
@@ -142,6 +147,11 @@ __device__ __forceinline__ void named_barrier_arrive(int id, int count) {
 __device__ __forceinline__ void named_barrier_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 __device__ __forceinline__ uint32_t atomic_add_acq_rel(uint32_t* p, uint32_t v) {
   uint32_t old;
   asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
@@ -182,8 +192,19 @@ constexpr int kProducerWarps = 4;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kGemvThreads = kConsumers + kProducerWarps * 32;
 constexpr int kGemvMaxRegs = 168;
+// After the start the producer warpgroup hands registers to the consumers:
+// 128 x 80 + 256 x 208 = 63,488 of the 384 x 168 = 64,512 the CTA is launched
+// with (per SM sub-partition: 2 x 32 x 208 + 32 x 80 = 15,872 <= 3 x 32 x 168).
+constexpr int kProducerRegs = 80;
+constexpr int kConsumerRegs = 208;
+static_assert(kProducerWarps * 32 * kProducerRegs + kConsumers * kConsumerRegs <= kGemvThreads * kGemvMaxRegs,
+              "register split exceeds the launch allocation");
 constexpr int kRowsPerProducerLane = kRows / (kProducerWarps * 32);
 constexpr uint32_t kSxaHole = 128;     // first pair-table hole row of the s X A^T staging
+// A CTA that ends its part of its first tile within this many steps of its
+// start counts that part at its next tile end instead (the previous kernel,
+// which zeroes the counters, may still be running that early).
+constexpr int64_t kDeferSteps = 3;
 
 template <int kNT, bool kQuad>   // kNT: n8 token tiles (1: M <= 8, 2: M <= 16); kQuad: K % 256 == 0
 __global__ void __maxnreg__(kGemvMaxRegs)
@@ -237,6 +258,16 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
   // Block constants of step p for tile rows lane + 32 j (j < 8), staged in the
   // free halves of the pair-table rows: slot s holds row r's four constants at
   // hole(32 s + r / 8, 16 (r mod 8)).
+  const uint32_t xbytes = 4u * static_cast<uint32_t>(m) * 128u;
+  // the loads of one stage: the code tile and the four activation boxes of step p
+  auto issue_stage = [&](Pos p, uint32_t st) {
+    mbar_arrive_expect_tx(&full[st], kCodeTile + xbytes);
+    const int col0 = p.step * kStepCols;
+    tma_load_2d(gptr(code_stage(st)), &cmap, col0 / 2, p.tile * kRows, &full[st]);
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+      tma_load_2d(gptr(xs0 + st * kXTile + b * kXBox), &xmap, col0 + b * 64, 0, &full[st]);
+  };
   if (threadIdx.x == kConsumers) {
     tma_prefetch_desc(&cmap);
     tma_prefetch_desc(&xmap);
@@ -248,6 +279,7 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
     fence_barrier_init();
   }
   if (warp >= kConsumerWarps) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
     // ------------------------------------------------ producer warps
     // Thread 0 of warp 8 streams the [256 rows x 128 bytes] code tile
     // (128B-swizzled) and the four [m x 64] activation boxes of each step into
@@ -330,7 +362,6 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
         sts128(hole(32u * slot + (r >> 3), (r & 7u) * 16u), c[0], c[1], c[2], c[3]);
       }
     };
-    const uint32_t xbytes = 4u * static_cast<uint32_t>(m) * 128u;
     Pos p = first;
     Pos p2 = advance(advance(first));
     RowConsts ra[kRowsPerProducerLane], rb[kRowsPerProducerLane];                // raw constants of steps it and it + 1
@@ -344,14 +375,7 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
       bool ok = true;
       if (lane == 0) ok = mbar_test_wait(&empty[ps], pph ^ 1u) || mbar_wait(&empty[ps], pph ^ 1u, a.err);
       if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
-      if (tma_thread) {
-        mbar_arrive_expect_tx(&full[ps], kCodeTile + xbytes);
-        const int col0 = p.step * kStepCols;
-        tma_load_2d(gptr(code_stage(ps)), &cmap, col0 / 2, p.tile * kRows, &full[ps]);
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-          tma_load_2d(gptr(xs0 + ps * kXTile + b * kXBox), &xmap, col0 + b * 64, 0, &full[ps]);
-      }
+      if (tma_thread) issue_stage(p, ps);
       write_consts(p, ra, ps);
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[ps]);   // the warp's constant stores are ordered before it
@@ -363,6 +387,7 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
     }
     return;
   }
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
   // pair table: entry (byte v, lane l) = {bf16(L[v >> 4]), bf16(L[v & 15])}, element order;
   // consumer thread v converts entry v once and writes its 32 copies
   {
@@ -546,11 +571,11 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
   };
   // Tile partials.  A CTA's share touches at most two tiles that other CTAs
   // share too, its first and its last; every tile inside the share lies in
-  // it alone.  At the end of its part of a tile a warp writes its fp32 partial
-  // to one of the CTA's two slots (plain stores, [cta][2][warp][lane][16]
-  // floats) and counts itself in the tile's per-warp counter; the warp whose
-  // arrival completes the count sums the slots of every CTA of the tile and
-  // finishes those 32 rows.
+  // it alone and is finished at once.  At the end of its part of a shared
+  // tile a warp writes its fp32 partial to one of the CTA's two slots (plain
+  // stores, [cta][2][warp][lane][16] floats) and counts itself in the tile's
+  // per-warp counter; the warp whose arrival completes the count sums the
+  // slots of every CTA of the tile in CTA order and finishes those 32 rows.
   auto shares_of = [&](int tile) -> int {
     const int64_t u0 = static_cast<int64_t>(tile) * steps;
     return static_cast<int>(owner_of(u0 + steps - 1, total, ctas) - owner_of(u0, total, ctas) + 1);
@@ -614,6 +639,49 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
     }
     finish(tile, v);
   };
+  // At the end of the share: when every other part of `tile` is already
+  // counted, this CTA is the last without counting itself; it adds the parts
+  // in CTA order with its own from registers (the sum the counting path
+  // forms) and finishes the tile.  Otherwise it returns false.
+  auto finish_if_complete = [&](int tile, const float (&own)[2][kNT][4]) -> bool {
+    const int shares = shares_of(tile);
+    uint32_t seen = 0;
+    if (lane == 0) seen = ld_acquire_u32(a.cnt + static_cast<int64_t>(tile) * kConsumerWarps + warp);
+    seen = __shfl_sync(0xFFFFFFFFu, seen, 0);
+    if (static_cast<int>(seen) + 1 != shares) return false;
+    float v[2][kNT][4];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int n = 0; n < kNT; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[i][n][e] = 0.0f;
+    const int64_t u0 = static_cast<int64_t>(tile) * steps;
+    const int64_t c0 = owner_of(u0, total, ctas);
+    for (int k = 0; k < shares; ++k) {
+      const int64_t c = c0 + k;
+      float4 q[2 * kNT];
+      if (c == blockIdx.x) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+          for (int n = 0; n < kNT; ++n) q[i * kNT + n] = make_float4(own[i][n][0], own[i][n][1], own[i][n][2], own[i][n][3]);
+      } else {
+        const float4* src = slot_ptr(c, bound(static_cast<int>(c), total, ctas) >= u0 ? 0 : 1);
+#pragma unroll
+        for (int f = 0; f < 2 * kNT; ++f) q[f] = __ldcg(src + f);
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int n = 0; n < kNT; ++n) {
+          const float4 w = q[i * kNT + n];
+          v[i][n][0] += w.x; v[i][n][1] += w.y; v[i][n][2] += w.z; v[i][n][3] += w.w;
+        }
+    }
+    finish(tile, v);
+    return true;
+  };
   // LoRA B rows of a tile into L2 ahead of its finish (lane (g, t) takes row
   // group t of its rows, one 128-byte line per 64 rank columns)
   auto prefetch_b = [&](int tile) {
@@ -634,10 +702,12 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
     for (int n = 0; n < kNT; ++n)
 #pragma unroll
       for (int e = 0; e < 4; ++e) y[i][n][e] = 0.0f;
-  // The first tile's partial goes to slot 0 at once; its count waits for the
-  // next tile boundary (or the end of the share), when the previous kernel
-  // (X A^T slices, zeroed counters) has surely finished, so the wait for it
-  // does not stall the stream.
+  // A first tile that ends within kDeferSteps steps of the start goes to slot 0
+  // at once and is counted at the next tile end (or the end of the share),
+  // when the previous kernel (X A^T slices, zeroed counters) has surely
+  // finished, so the wait for it does not stall the stream.  A later first
+  // tile end waits for that kernel (long done by then) and counts at once, so
+  // that the share's end finds it counted.
   int pending = -1;
   bool dep_done = false;
 
@@ -703,13 +773,15 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
     }
 
     if (pos.step == steps - 1 || it == n_mine - 1) {
-      // end of this CTA's share of the tile: its partial goes to the slot (0 for
-      // the share's first tile, else 1; a tile inside the share is counted and
-      // finished at once, so slot 1 is free again for the next one)
-      put_slot(pos.tile == first.tile ? 0 : 1, y);
-      if (it != n_mine - 1) prefetch_b(pos.tile + 1);
-      if (!dep_done && pending < 0 && it != n_mine - 1) {
-        pending = pos.tile;                                   // counted later
+      // end of this CTA's part of the tile
+      const bool last = it == n_mine - 1;
+      const int shares = shares_of(pos.tile);
+      if (!last) prefetch_b(pos.tile + 1);
+      if (!dep_done && pending < 0 && !last && shares > 1 && it < kDeferSteps) {
+        // so early that the previous kernel (X A^T slices, zeroed counters) may
+        // still run: the partial waits in slot 0 and is counted later
+        put_slot(0, y);
+        pending = pos.tile;
       } else {
         if (!dep_done) {
           grid_dependency_wait();
@@ -719,11 +791,19 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
           if (lane == 0) mbar_arrive(xa_bar);
           if (!mbar_test_wait(xa_bar, 0) && !mbar_wait(xa_bar, 0, a.err)) { alive = false; break; }
         }
-        for (int k = 0; k < 2; ++k) {
-          const int tl = k == 0 ? pending : pos.tile;
-          if (tl >= 0) arrive(tl, y);
+        if (pending >= 0) {
+          float v[2][kNT][4];
+          arrive(pending, v);
+          pending = -1;
         }
-        pending = -1;
+        if (shares == 1) {
+          finish(pos.tile, y);                                // no other CTA holds a part of it
+        } else if (!(last && finish_if_complete(pos.tile, y))) {
+          // slot 0 for the share's first tile, else 1 (a tile inside the share
+          // is finished at once, so slot 1 is free again for the next one)
+          put_slot(pos.tile == first.tile ? 0 : 1, y);
+          arrive(pos.tile, y);
+        }
       }
 #pragma unroll
       for (int i = 0; i < 2; ++i)
@@ -741,9 +821,11 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
 // Partial X A^T and the zeroed tile counters of k_gemv.  CTA (c, sp) computes
 // LoRA columns 4c .. 4c + 3 for every token over the sp-th of nsplit slices of
 // K and writes them to part[sp] (no atomics, so nothing needs zeroing); k_gemv
-// sums the slices when it first finishes a tile.  Each of the 64 threads takes
-// 8-column chunks a block stride apart; the CTA reduces with warp shuffles and
-// one exchange through shared memory.  k_gemv, launched as the programmatic
+// sums the slices when it first finishes a tile.  The CTA has a thread per
+// 8-column chunk of its slice (a grid-stride loop covers longer slices), so
+// the whole grid waits for about one load latency; warps reduce with shuffles
+// and the warps' sums are added in warp order through shared memory, so the
+// result does not depend on timing.  k_gemv, launched as the programmatic
 // dependent of this grid, waits for it only before it first counts a tile.
 // The four A rows' 8 columns of chunk ch, unpacked.
 __device__ __forceinline__ void load_a_rows(const uint16_t* __restrict__ A, int j0, int r, int64_t kw,
@@ -757,15 +839,17 @@ __device__ __forceinline__ void load_a_rows(const uint16_t* __restrict__ A, int 
   }
 }
 
+constexpr int kXaMaxThreads = 256;
+
 // kMulti: every token has its own adapter (A + idx[i] * a_stride); its A rows
 // are loaded per token.  Tokens without a valid adapter accumulate nothing.
 template <int kMaxM, bool kMulti>
-__global__ void __launch_bounds__(64, 8)
+__global__ void __launch_bounds__(kXaMaxThreads)
 k_xa_zero(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A, int64_t m, int64_t kw, int r,
           float* __restrict__ part, int64_t ld, float4* __restrict__ zero4, int64_t n4,
           const int32_t* __restrict__ idx, int n_adapters, int64_t a_stride, uint32_t* err) {
   launch_dependents();
-  __shared__ float s_red[4 * kMaxM];
+  __shared__ float s_red[kXaMaxThreads / 32][4 * kMaxM];
   const int mi = static_cast<int>(m);
   const int j0 = blockIdx.x * 4;
   const int64_t nch = kw / 8;
@@ -788,11 +872,11 @@ k_xa_zero(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A, int64_
   for (int64_t ch = c_beg + threadIdx.x; ch < c_end; ch += blockDim.x) {
     float af[4][8];
     if constexpr (!kMulti) {
-      load_a_rows(A, j0, r, kw, ch, af);     // shared by every token
-      uint4 xv[kMaxM];
+      uint4 xv[kMaxM];                       // every load of the chunk issued before any use
 #pragma unroll
       for (int i = 0; i < kMaxM; ++i)
         xv[i] = i < mi ? __ldg(reinterpret_cast<const uint4*>(X + i * kw) + ch) : make_uint4(0u, 0u, 0u, 0u);
+      load_a_rows(A, j0, r, kw, ch, af);     // shared by every token
 #pragma unroll
       for (int i = 0; i < kMaxM; ++i) {
         const float xf[8] = {bf16_lo(xv[i].x), bf16_hi(xv[i].x), bf16_lo(xv[i].y), bf16_hi(xv[i].y),
@@ -819,6 +903,7 @@ k_xa_zero(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A, int64_
     }
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = static_cast<int>(blockDim.x >> 5);
 #pragma unroll
   for (int c = 0; c < 4; ++c)
 #pragma unroll
@@ -826,25 +911,25 @@ k_xa_zero(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A, int64_
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) acc[c][i] += __shfl_xor_sync(0xFFFFFFFFu, acc[c][i], o);
     }
-  if (warp == 1 && lane == 0) {
+  if (lane == 0) {
 #pragma unroll
     for (int c = 0; c < 4; ++c)
 #pragma unroll
-      for (int i = 0; i < kMaxM; ++i) s_red[c * kMaxM + i] = acc[c][i];
+      for (int i = 0; i < kMaxM; ++i) s_red[warp][c * kMaxM + i] = acc[c][i];
   }
   __syncthreads();
-  if (warp == 0 && lane == 0) {
-    float* dst = part + static_cast<int64_t>(blockIdx.y) * 16 * ld;
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-#pragma unroll
-      for (int i = 0; i < kMaxM; ++i)
-        if (i < mi && j0 + c < r) dst[i * ld + j0 + c] = acc[c][i] + s_red[c * kMaxM + i];
+  // thread e < 4 kMaxM adds output e over the warps in order
+  const int e = static_cast<int>(threadIdx.x);
+  if (e < 4 * kMaxM) {
+    const int c = e / kMaxM, i = e - (e / kMaxM) * kMaxM;
+    float v = 0.0f;
+    for (int w = 0; w < nwarps; ++w) v += s_red[w][e];
+    if (i < mi && j0 + c < r) part[(static_cast<int64_t>(blockIdx.y) * 16 + i) * ld + j0 + c] = v;
   }
   const int64_t nthreads = static_cast<int64_t>(gridDim.x) * gridDim.y * blockDim.x;
   const int64_t gtid = (static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x;
   const float4 z = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  for (int64_t e = gtid; e < n4; e += nthreads) zero4[e] = z;
+  for (int64_t q = gtid; q < n4; q += nthreads) zero4[q] = z;
 }
 
 cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, void** args) {
@@ -901,35 +986,50 @@ int64_t gemv_slot_floats(int64_t m_tiles, int64_t steps) {
 }
 
 template <bool kMulti>
-void launch_xa_zero_t(dim3 grid, const uint16_t* X, const uint16_t* A, int64_t m, int64_t kw, int r,
-                      float* part, int64_t ld, float4* z4, int64_t n4, const int32_t* idx, int n_ad,
+void launch_xa_zero_t(dim3 grid, unsigned threads, const uint16_t* X, const uint16_t* A, int64_t m, int64_t kw,
+                      int r, float* part, int64_t ld, float4* z4, int64_t n4, const int32_t* idx, int n_ad,
                       int64_t a_stride, uint32_t* err, cudaStream_t stream) {
-  if (m <= 1) k_xa_zero<1, kMulti><<<grid, 64, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4, idx, n_ad, a_stride, err);
-  else if (m <= 4) k_xa_zero<4, kMulti><<<grid, 64, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4, idx, n_ad, a_stride, err);
-  else if (m <= 8) k_xa_zero<8, kMulti><<<grid, 64, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4, idx, n_ad, a_stride, err);
-  else k_xa_zero<16, kMulti><<<grid, 64, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4, idx, n_ad, a_stride, err);
+  if (m <= 1)
+    k_xa_zero<1, kMulti><<<grid, threads, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4, idx, n_ad, a_stride, err);
+  else if (m <= 4)
+    k_xa_zero<4, kMulti><<<grid, threads, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4, idx, n_ad, a_stride, err);
+  else if (m <= 8)
+    k_xa_zero<8, kMulti><<<grid, threads, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4, idx, n_ad, a_stride, err);
+  else
+    k_xa_zero<16, kMulti><<<grid, threads, 0, stream>>>(X, A, m, kw, r, part, ld, z4, n4, idx, n_ad, a_stride, err);
 }
 
 cudaError_t launch_xa_zero(const uint16_t* X, const uint16_t* A, int64_t m, int64_t kw, int r, float* part,
                            int64_t ld, int splits, float* zero, int64_t n_zero, const int32_t* adapter_idx,
                            int n_adapters, int64_t a_stride, uint32_t* err, cudaStream_t stream) {
   const dim3 grid(static_cast<unsigned>((r + 3) / 4), static_cast<unsigned>(splits));
+  // a thread per chunk of the longest slice, in whole warps (at most
+  // kXaMaxThreads): a thread that loads two chunks at once is slower
+  const int64_t per_split = (kw / 8 + splits - 1) / splits;
+  int64_t threads = (per_split + 31) / 32 * 32;
+  if (threads > kXaMaxThreads) threads = kXaMaxThreads;
+  if (threads < 64) threads = 64;
   float4* z4 = reinterpret_cast<float4*>(zero);
   const int64_t n4 = n_zero / 4;
   if (adapter_idx)
-    launch_xa_zero_t<true>(grid, X, A, m, kw, r, part, ld, z4, n4, adapter_idx, n_adapters, a_stride, err, stream);
+    launch_xa_zero_t<true>(grid, static_cast<unsigned>(threads), X, A, m, kw, r, part, ld, z4, n4, adapter_idx,
+                           n_adapters, a_stride, err, stream);
   else
-    launch_xa_zero_t<false>(grid, X, A, m, kw, r, part, ld, z4, n4, nullptr, 1, 0, err, stream);
+    launch_xa_zero_t<false>(grid, static_cast<unsigned>(threads), X, A, m, kw, r, part, ld, z4, n4, nullptr, 1,
+                            0, err, stream);
   return cudaGetLastError();
 }
 
 int xa_splits_for(int r, int64_t kw) {
+  // about 128 CTAs with a thread per 8-column chunk; more slices (up to the
+  // most k_gemv sums) and threads when K is longer
   const int groups = (r + 3) / 4;
-  int s = 128 / groups;                       // about 128 CTAs in all
-  const int64_t max_by_k = (kw / 8) / 64;     // at least one chunk per thread
-  if (s > max_by_k) s = static_cast<int>(max_by_k);
+  const int64_t want = (kw / 8 + 127) / 128;  // slices of 128 chunks
+  int64_t s = 128 / groups;
+  if (s < want) s = want;
   if (s > kMaxXaSplits) s = kMaxXaSplits;
-  return s < 1 ? 1 : s;
+  if (s > (kw / 8) / 32) s = (kw / 8) / 32;   // at least a warp of chunks per slice
+  return s < 1 ? 1 : static_cast<int>(s);
 }
 
 cudaError_t launch_gemv(const GemvArgs& args, const CUtensorMap& codes_map, const CUtensorMap& x_map,
