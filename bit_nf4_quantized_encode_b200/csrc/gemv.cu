@@ -477,6 +477,22 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
       }
     }
   };
+  // Per-token adapters, read once: lane j < m holds token j's adapter (-1 for
+  // none or out of range), and bit j of first_use marks the token that uses
+  // its adapter first, so the adapters in use are visited in order of first
+  // use without reading the index array again.
+  int my_ad = -1;
+  uint32_t first_use = 1u;                          // one pass for the single adapter
+  if (a.adapter_idx != nullptr) {
+    if (lane < m) my_ad = __ldg(a.adapter_idx + lane);
+    if (my_ad >= a.n_adapters) my_ad = -1;
+    const uint32_t same = __match_any_sync(0xFFFFFFFFu, my_ad);
+    const bool first = my_ad >= 0 && (same & ((1u << lane) - 1u)) == 0;
+    first_use = __ballot_sync(0xFFFFFFFFu, first);
+  }
+  auto for_each_adapter = [&](auto&& fn) {
+    for (uint32_t mk = first_use; mk != 0; mk &= mk - 1u) fn(__shfl_sync(0xFFFFFFFFu, my_ad, __ffs(mk) - 1));
+  };
   // The LoRA up-projection s (X A^T) B^T of one adapter added to this lane's
   // fp32 sums with warp MMAs: A operand = rows of that adapter's B (lb), B
   // operand = the staged bf16(s X A^T) of the tokens `use` selects (the other
@@ -523,18 +539,6 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
       }
     }
   };
-  // The adapters of a call with per-token adapters, each once (in order of
-  // first use); fn(adapter) is called for each.  Warp-uniform: every lane
-  // reads the same indices.
-  auto for_each_adapter = [&](auto&& fn) {
-    for (int j = 0; j < m; ++j) {
-      const int aj = __ldg(a.adapter_idx + j);
-      if (aj < 0 || aj >= a.n_adapters) continue;
-      bool first = true;
-      for (int k2 = 0; k2 < j; ++k2) first = first && __ldg(a.adapter_idx + k2) != aj;
-      if (first) fn(aj);
-    }
-  };
   // Y rows of tile `tile` for this lane from its fp32 sums: add the LoRA term
   // (one pass per adapter in use) and store bf16.
   auto finish = [&](int tile, float (&acc)[2][kNT][4]) {
@@ -545,13 +549,10 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
       for (int n = 0; n < kNT; ++n) all[n] = true;
       lora_pass(tile, a.lora_b, all, acc);
     } else {
-      int tok_ad[kNT];                              // the adapter of this lane's token 8n + g
-#pragma unroll
-      for (int n = 0; n < kNT; ++n) tok_ad[n] = 8 * n + g < m ? __ldg(a.adapter_idx + 8 * n + g) : -1;
       for_each_adapter([&](int ad) {
         bool use[kNT];
 #pragma unroll
-        for (int n = 0; n < kNT; ++n) use[n] = tok_ad[n] == ad;
+        for (int n = 0; n < kNT; ++n) use[n] = __shfl_sync(0xFFFFFFFFu, my_ad, 8 * n + g) == ad;
         lora_pass(tile, a.lora_b + static_cast<int64_t>(ad) * a.b_stride, use, acc);
       });
     }
@@ -685,9 +686,12 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
   // LoRA B rows of a tile into L2 ahead of its finish (lane (g, t) takes row
   // group t of its rows, one 128-byte line per 64 rank columns)
   auto prefetch_b = [&](int tile) {
+    // every lane walks the adapters (their list is shuffled across the warp);
+    // only lanes with a row in the weight prefetch
     const int64_t row = static_cast<int64_t>(tile) * kRows + warp * 32 + 8 * t + pg;
-    if (row >= a.nw) return;
+    const bool in_w = row < a.nw;
     auto rows_of = [&](const uint16_t* lb) {
+      if (!in_w) return;
       for (int grp = 0; grp < a.lora_steps; ++grp)
         asm volatile("prefetch.global.L2 [%0];" ::"l"(lb + row * a.r + grp * 64));
     };
