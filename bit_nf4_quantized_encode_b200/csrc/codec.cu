@@ -53,6 +53,38 @@ __device__ __forceinline__ uint32_t exact_code(float n, const float* s_thr, cons
   return s_base[u] + (n >= s_thr[u] ? 1u : 0u);
 }
 
+// Packed pairs of floats (sm_100 f32x2 arithmetic, round to nearest even;
+// each lane of the pair rounds exactly as the scalar operation does).
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t v;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+  return v;
+}
+__device__ __forceinline__ void unpack_f32x2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// Per half: the larger of |a| and |b| as its magnitude (bf16 pairs).
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 __device__ __forceinline__ float nan_min_abs(float m, float d) {
   float r;
   asm("{\n\t.reg .f32 t;\n\tabs.f32 t, %2;\n\tmin.NaN.f32 %0, %1, t;\n\t}" : "=f"(r) : "f"(m), "f"(d));
@@ -94,9 +126,12 @@ __global__ void __launch_bounds__(256) k_encode(const uint16_t* __restrict__ w, 
       x[2 * k] = bf16_lo(wd[k]);
       x[2 * k + 1] = bf16_hi(wd[k]);
     }
-    float amax = 0.0f;
+    // |x| max on the packed pairs: the magnitude of max.xorsign.abs is the
+    // larger magnitude, exactly (NaN weights are outside the encoder's domain)
+    uint32_t pmax = 0u;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    for (int k = 0; k < 8; ++k) pmax = bf16x2_absmax(pmax, wd[k]);
+    float amax = fmaxf(fabsf(bf16_lo(pmax)), fabsf(bf16_hi(pmax)));
     amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
     if (!on) return;
@@ -107,22 +142,30 @@ __global__ void __launch_bounds__(256) k_encode(const uint16_t* __restrict__ w, 
       bool exact = !fast_ok || !(amax >= 0x1.0p-125f) || !(amax <= 3.0e38f);
       if (!exact) {
         const float r = __frcp_rn(amax);
+        const uint64_t r2 = pack_f32x2(r, r);
+        const uint64_t c16 = pack_f32x2(16.0f, 16.0f), cbias = pack_f32x2(8388624.0f, 8388624.0f);
         float m = INFINITY;
         uint32_t pk[2] = {0u, 0u};
-        // nibble order: element 2j -> high nibble of byte j; shift-add from byte 3 down
+        // nibble order: element 2j -> high nibble of byte j; shift-add from byte 3 down.
+        // The two elements of a word go through the same packed multiply, fma
+        // and subtraction (each rounded like its scalar form).
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
           for (int jj = 3; jj >= 0; --jj) {
+            const uint64_t n2 = mul_f32x2(pack_f32x2(x[8 * h + 2 * jj], x[8 * h + 2 * jj + 1]), r2);
+            float f[2];
+            unpack_f32x2(fma_f32x2(n2, c16, cbias), f[0], f[1]);
+            uint32_t tw[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+              asm("ld.shared.b32 %0, [%1];" : "=r"(tw[e]) : "r"(fast_tbl + (__float_as_uint(f[e]) & 63u) * 4u));
+            float d[2];
+            unpack_f32x2(sub_f32x2(n2, pack_f32x2(__uint_as_float(tw[0]), __uint_as_float(tw[1]))), d[0], d[1]);
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-              const float n = __fmul_rn(x[8 * h + 2 * jj + e], r);
-              const uint32_t u = __float_as_uint(__fmaf_rn(n, 16.0f, 8388624.0f)) & 63u;
-              uint32_t tw;
-              asm("ld.shared.b32 %0, [%1];" : "=r"(tw) : "r"(fast_tbl + u * 4u));
-              const float d = __fsub_rn(n, __uint_as_float(tw));
-              m = nan_min_abs(m, d);
-              const uint32_t code = (tw & 31u) - (__float_as_uint(d) >> 31);
+              m = nan_min_abs(m, d[e]);
+              const uint32_t code = (tw[e] & 31u) - (__float_as_uint(d[e]) >> 31);
               pk[h] = (pk[h] << 4) + code;
             }
           }
