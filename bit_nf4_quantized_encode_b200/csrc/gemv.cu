@@ -650,6 +650,7 @@ k_gemv(const GemvArgs a, const __grid_constant__ CUtensorMap cmap,
     if (lane == 0) seen = ld_acquire_u32(a.cnt + static_cast<int64_t>(tile) * kConsumerWarps + warp);
     seen = __shfl_sync(0xFFFFFFFFu, seen, 0);
     if (static_cast<int>(seen) + 1 != shares) return false;
+    __syncwarp();      // lane 0's acquire is ordered before every lane's slot reads
     float v[2][kNT][4];
 #pragma unroll
     for (int i = 0; i < 2; ++i)
