@@ -88,6 +88,12 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void* p, uint64_t pol) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p), "l"(pol));
   return v;
 }
+// 32 bytes in one request (sm_100 256-bit load); p must be 32-byte aligned.
+__device__ __forceinline__ void ldg_nc_v8(const void* p, uint64_t pol, uint4& lo, uint4& hi) {
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8], %9;"
+               : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+               : "l"(p), "l"(pol));
+}
 
 // Prefetched inputs of one dequant task.
 struct DqLoad {
@@ -97,8 +103,12 @@ struct DqLoad {
   bool valid;
 };
 
+// A block's 32 code bytes start at a multiple of 32 bytes of the code array,
+// so with a 32-byte aligned array they take one 256-bit load (one L2 request
+// per row instead of two; measured +3% on the fused kernel), else two.
 template <int kDir>
-__device__ __forceinline__ DqLoad dq_load(const FusedArgs& a, int m0, int kstep, int t, uint64_t pol) {
+__device__ __forceinline__ DqLoad dq_load(const FusedArgs& a, int m0, int kstep, int t, uint64_t pol,
+                                          bool codes32) {
   DqLoad d;
   int64_t n, kcol;
   if (kDir == 0) {              // forward: task = W row m0 + t, block kstep
@@ -112,8 +122,12 @@ __device__ __forceinline__ DqLoad dq_load(const FusedArgs& a, int m0, int kstep,
   if (d.valid) {
     const int64_t e = n * a.kw + kcol;                 // first weight of the block
     const uint8_t* p = a.codes + (e >> 1);
-    d.c0 = ldg_nc_v4(p, pol);
-    d.c1 = ldg_nc_v4(p + 16, pol);
+    if (codes32) {
+      ldg_nc_v8(p, pol, d.c0, d.c1);
+    } else {
+      d.c0 = ldg_nc_v4(p, pol);
+      d.c1 = ldg_nc_v4(p + 16, pol);
+    }
     const int64_t blk = e >> 6;
     if (a.absf) {                 // no double quantization: the constant itself
       d.q = 0;
@@ -240,6 +254,7 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
     const bool plain = a.absf != nullptr;
     const float mu = plain ? 0.0f : __ldg(a.mean);
     const uint64_t codes_pol = l2_evict_last_policy();
+    const bool codes32 = (reinterpret_cast<uintptr_t>(a.codes) & 31u) == 0;
     uint32_t gctr = 0;
     bool alive = true;
     for (int u = blockIdx.x; u < nunits && alive; u += gridDim.x) {
@@ -247,12 +262,13 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
       const int m0 = w.mt * 128;
       int j = static_cast<int>((static_cast<uint32_t>(group) - gctr) & (kDequantGroups - 1));
       DqLoad next;
-      if (j < w.kmain) next = dq_load<kDir>(a, m0, w.kbeg + j, t, codes_pol);
+      if (j < w.kmain) next = dq_load<kDir>(a, m0, w.kbeg + j, t, codes_pol, codes32);
       for (; j < w.nk; j += kDequantGroups) {
         const uint32_t it = gctr + j;
         const uint32_t stage = it % kStages, phase = (it / kStages) & 1u;
         const DqLoad cur = next;
-        if (j + kDequantGroups < w.kmain) next = dq_load<kDir>(a, m0, w.kbeg + j + kDequantGroups, t, codes_pol);
+        if (j + kDequantGroups < w.kmain)
+          next = dq_load<kDir>(a, m0, w.kbeg + j + kDequantGroups, t, codes_pol, codes32);
         if (!mbar_wait(&empty[stage], phase ^ 1u, a.err)) { alive = false; break; }
         const uint32_t sA = smem0 + stage * kStageBytes;
         if (j < w.kmain) dq_store<kDir>(sA, t, cur, mu, plain, a.cb);
