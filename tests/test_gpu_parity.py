@@ -308,3 +308,32 @@ def test_results_are_bit_reproducible(qb, n, k, m):
         if name == "dX" and m <= 16:
             continue                                  # split-K fp32 atomics at 16 tokens or fewer
         assert torch.equal(a, b), f"{name} differs between two identical calls ({n}x{k}, m={m})"
+
+
+@pytest.mark.parametrize("m", [64, 8])
+def test_codes_at_a_16_byte_offset_give_identical_results(qb, m):
+    """The fused kernel loads a block's 32 code bytes in one 256-bit load when
+    the code array is 32-byte aligned and in two 128-bit loads otherwise; both
+    paths give the same bits."""
+    import dataclasses
+    n, k, r = 392, 640, 64
+    W = workloads.weight((n, k), proj=3).cuda()
+    qt = qb.qlora_quantize_nf4_dq(W)
+    base = torch.empty(qt.codes.numel() + 32, dtype=torch.uint8, device="cuda")
+    off = 16 - base.data_ptr() % 32 if base.data_ptr() % 32 <= 16 else 48 - base.data_ptr() % 32
+    codes16 = base[off:off + qt.codes.numel()]
+    assert codes16.data_ptr() % 32 == 16
+    codes16.copy_(qt.codes)
+    qt16 = dataclasses.replace(qt, codes=codes16)
+    X = workloads.activations(m, k, 3).cuda()
+    dY = workloads.grad_output(m, n, 3).cuda()
+    A, B = workloads.lora_a(r, k, 3).cuda(), workloads.lora_b(n, r, 3).cuda()
+    outs = []
+    for t in (qt, qt16):
+        Y, XA = qb.qlora_linear_fwd(t, X, A, B, 0.25)
+        dX, dA, dB = qb.qlora_linear_bwd(t, X, dY, A, B, 0.25, XA=XA)
+        outs.append((Y, dX, dA, dB))
+    torch.cuda.synchronize()
+    assert qb.qlora_read_device_errors() == 0
+    for a, b, name in zip(outs[0], outs[1], ("Y", "dX", "dA", "dB")):
+        assert torch.equal(a, b), name
