@@ -43,12 +43,22 @@ std::mutex g_mu;
 std::atomic<uint64_t> g_launches{0};
 thread_local cudaEvent_t t_gemm_start = nullptr, t_gemm_stop = nullptr;
 
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch_bytes,
+                 uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
+
 cudaError_t fused_timed(FusedDir dir, int bn, const FusedArgs& fa, const CUtensorMap& act,
                         const CUtensorMap& lora, int num_sms, cudaStream_t cs) {
+  // the dequant groups' code tiles: forward 128 rows x 32 bytes (one block of
+  // each row), backward 64 rows x 64 bytes (two blocks of each row)
+  CUtensorMap codes_map;
+  const bool fwd = dir == FusedDir::kFwd;
+  if (!make_map_u8(&codes_map, fa.codes, static_cast<uint64_t>(fa.kw / 2), static_cast<uint64_t>(fa.nw),
+                   static_cast<uint64_t>(fa.kw / 2), fwd ? 32 : 64, fwd ? 128 : 64, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
   cudaEvent_t e0 = t_gemm_start, e1 = t_gemm_stop;
   t_gemm_start = t_gemm_stop = nullptr;
   if (e0 && cudaEventRecord(e0, cs) != cudaSuccess) return cudaErrorUnknown;
-  cudaError_t e = counted(launch_fused(dir, bn, fa, act, lora, num_sms, cs));
+  cudaError_t e = counted(launch_fused(dir, bn, fa, act, lora, codes_map, num_sms, cs));
   if (e == cudaSuccess && e1) e = cudaEventRecord(e1, cs);
   return e;
 }

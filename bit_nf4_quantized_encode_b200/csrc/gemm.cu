@@ -37,8 +37,13 @@ constexpr int kFusedThreads = (kMmaWarp + 1) * 32;
 __host__ __device__ constexpr int fused_stages(int bn) { return bn >= 128 ? 4 : 8; }
 static_assert(kDequantGroups == 4, "stage ring and group rotation assume four groups");
 __host__ __device__ constexpr int fused_tmem_cols(int bn) { return 2 * bn < 32 ? 32 : 2 * bn; }
+// Packed codes of one dequant task set (4 KB: 128 rows x 32 B forward, 64 rows
+// x 64 B backward), loaded by TMA into one of two slots per dequant group.
+constexpr int kCodeSlotBytes = 4096;
+constexpr int kCodeSlots = 2 * kDequantGroups;
 __host__ __device__ constexpr size_t fused_smem_bytes(int bn) {
-  return 1024 + static_cast<size_t>(fused_stages(bn)) * (kATileBytes + bn * 128) + 512;
+  return 1024 + static_cast<size_t>(fused_stages(bn)) * (kATileBytes + bn * 128) +
+         static_cast<size_t>(kCodeSlots) * kCodeSlotBytes + 512;
 }
 
 // Work unit -> (m-tile, token tile, split) and its k-step range.  Units run in
@@ -95,6 +100,13 @@ __device__ __forceinline__ void ldg_nc_v8(const void* p, uint64_t pol, uint4& lo
                : "l"(p), "l"(pol));
 }
 
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr) : "memory");
+  return v;
+}
+
 // Prefetched inputs of one dequant task.
 struct DqLoad {
   uint4 c0, c1;        // 64 packed codes (32 bytes)
@@ -107,8 +119,7 @@ struct DqLoad {
 // so with a 32-byte aligned array they take one 256-bit load (one L2 request
 // per row instead of two; measured +3% on the fused kernel), else two.
 template <int kDir>
-__device__ __forceinline__ DqLoad dq_load(const FusedArgs& a, int m0, int kstep, int t, uint64_t pol,
-                                          bool codes32) {
+__device__ __forceinline__ DqLoad dq_load(const FusedArgs& a, int m0, int kstep, int t, uint64_t pol) {
   DqLoad d;
   int64_t n, kcol;
   if (kDir == 0) {              // forward: task = W row m0 + t, block kstep
@@ -121,13 +132,7 @@ __device__ __forceinline__ DqLoad dq_load(const FusedArgs& a, int m0, int kstep,
   d.valid = (n < a.nw) && (kcol < a.kw);
   if (d.valid) {
     const int64_t e = n * a.kw + kcol;                 // first weight of the block
-    const uint8_t* p = a.codes + (e >> 1);
-    if (codes32) {
-      ldg_nc_v8(p, pol, d.c0, d.c1);
-    } else {
-      d.c0 = ldg_nc_v4(p, pol);
-      d.c1 = ldg_nc_v4(p + 16, pol);
-    }
+    (void)pol;
     const int64_t blk = e >> 6;
     if (a.absf) {                 // no double quantization: the constant itself
       d.q = 0;
@@ -200,7 +205,7 @@ __device__ __forceinline__ void lora_store(const FusedArgs& a, uint32_t sA, int 
 template <int kDir, int kBN>
 __global__ void __launch_bounds__(kFusedThreads, 1)
 k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
-        const __grid_constant__ CUtensorMap lora_act) {
+        const __grid_constant__ CUtensorMap lora_act, const __grid_constant__ CUtensorMap codes_map) {
   constexpr int kStages = fused_stages(kBN);
   constexpr int kBTileBytes = kBN * 128;
   constexpr int kStageBytes = kATileBytes + kBTileBytes;
@@ -210,13 +215,15 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem0 = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem_gen = smem_raw + (smem0 - smem_u32(smem_raw));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_gen + kStages * kStageBytes);
+  const uint32_t code0 = smem0 + kStages * kStageBytes;     // kCodeSlots code slots
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_gen + kStages * kStageBytes + kCodeSlots * kCodeSlotBytes);
   uint64_t* full_a = bars;                   // [kStages] dequant -> MMA (128 arrivals)
   uint64_t* full_b = bars + kStages;         // [kStages] TMA -> MMA (tx bytes)
   uint64_t* empty = bars + 2 * kStages;      // [kStages] MMA -> producers (commit)
   uint64_t* acc_full = bars + 3 * kStages;   // [2] MMA -> epilogue (commit)
   uint64_t* acc_empty = acc_full + 2;        // [2] epilogue -> MMA (128 arrivals)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* code_full = acc_empty + 2;       // [kCodeSlots] code TMA -> dequant group (tx bytes)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(code_full + kCodeSlots);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -232,6 +239,7 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
     }
+    for (int c = 0; c < kCodeSlots; ++c) mbar_init(&code_full[c], 1);
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
@@ -241,6 +249,7 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
   if (warp == kTmaWarp && lane == 0) {
     tma_prefetch_desc(&act);
     tma_prefetch_desc(&lora_act);
+    tma_prefetch_desc(&codes_map);
   }
   tc_fence_before();
   __syncthreads();
@@ -254,7 +263,18 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
     const bool plain = a.absf != nullptr;
     const float mu = plain ? 0.0f : __ldg(a.mean);
     const uint64_t codes_pol = l2_evict_last_policy();
-    const bool codes32 = (reinterpret_cast<uintptr_t>(a.codes) & 31u) == 0;
+    // The group's code tiles come by TMA into two slots, one task ahead.  A
+    // slot is refilled only after this thread's wait on `empty` for the current
+    // task, which implies every thread of the group has finished the task
+    // before it, the last reader of that slot.
+    uint32_t ci = 0;                          // code tasks of this group so far
+    auto issue_codes = [&](uint32_t c, int m0, int kstep) {
+      const int slot = group * 2 + static_cast<int>(c & 1u);
+      mbar_arrive_expect_tx(&code_full[slot], kCodeSlotBytes);
+      uint8_t* dst = smem_gen + kStages * kStageBytes + slot * kCodeSlotBytes;
+      if (kDir == 0) tma_load_2d(dst, &codes_map, kstep * 32, m0, &code_full[slot]);
+      else tma_load_2d(dst, &codes_map, m0 / 2, kstep * 64, &code_full[slot]);
+    };
     uint32_t gctr = 0;
     bool alive = true;
     for (int u = blockIdx.x; u < nunits && alive; u += gridDim.x) {
@@ -262,17 +282,29 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
       const int m0 = w.mt * 128;
       int j = static_cast<int>((static_cast<uint32_t>(group) - gctr) & (kDequantGroups - 1));
       DqLoad next;
-      if (j < w.kmain) next = dq_load<kDir>(a, m0, w.kbeg + j, t, codes_pol, codes32);
+      if (j < w.kmain) {
+        next = dq_load<kDir>(a, m0, w.kbeg + j, t, codes_pol);
+        if (t == 0) issue_codes(ci, m0, w.kbeg + j);
+      }
       for (; j < w.nk; j += kDequantGroups) {
         const uint32_t it = gctr + j;
         const uint32_t stage = it % kStages, phase = (it / kStages) & 1u;
-        const DqLoad cur = next;
-        if (j + kDequantGroups < w.kmain)
-          next = dq_load<kDir>(a, m0, w.kbeg + j + kDequantGroups, t, codes_pol, codes32);
+        DqLoad cur = next;
+        if (j + kDequantGroups < w.kmain) next = dq_load<kDir>(a, m0, w.kbeg + j + kDequantGroups, t, codes_pol);
         if (!mbar_wait(&empty[stage], phase ^ 1u, a.err)) { alive = false; break; }
+        if (t == 0 && j + kDequantGroups < w.kmain) issue_codes(ci + 1, m0, w.kbeg + j + kDequantGroups);
         const uint32_t sA = smem0 + stage * kStageBytes;
-        if (j < w.kmain) dq_store<kDir>(sA, t, cur, mu, plain, a.cb);
-        else lora_store<kDir>(a, sA, m0, j - w.kmain, t);
+        if (j < w.kmain) {
+          const int slot = group * 2 + static_cast<int>(ci & 1u);
+          if (!mbar_wait(&code_full[slot], (ci >> 1) & 1u, a.err)) { alive = false; break; }
+          const uint32_t src = code0 + slot * kCodeSlotBytes + static_cast<uint32_t>(t) * 32u;
+          cur.c0 = lds_v4(src);
+          cur.c1 = lds_v4(src + 16);
+          ++ci;
+          dq_store<kDir>(sA, t, cur, mu, plain, a.cb);
+        } else {
+          lora_store<kDir>(a, sA, m0, j - w.kmain, t);
+        }
         fence_proxy_async_smem();
         mbar_arrive(&full_a[stage]);
       }
@@ -454,27 +486,28 @@ cudaError_t ensure_smem_attr(K kernel, size_t bytes, std::atomic<uint64_t>& done
 
 template <int kDir, int kBN>
 cudaError_t launch_fused_t(const FusedArgs& args, const CUtensorMap& act, const CUtensorMap& lora_act,
-                           int num_sms, cudaStream_t stream) {
+                           const CUtensorMap& codes_map, int num_sms, cudaStream_t stream) {
   static std::atomic<uint64_t> attr_done{0};
   const size_t smem = fused_smem_bytes(kBN);
   cudaError_t e = ensure_smem_attr(k_fused<kDir, kBN>, smem, attr_done);
   if (e != cudaSuccess) return e;
   const int nunits = args.m_tiles * args.t_tiles * args.splits;
   const int grid = nunits < num_sms ? nunits : num_sms;
-  k_fused<kDir, kBN><<<grid, kFusedThreads, smem, stream>>>(args, act, lora_act);
+  k_fused<kDir, kBN><<<grid, kFusedThreads, smem, stream>>>(args, act, lora_act, codes_map);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_fused(FusedDir dir, int token_tile, const FusedArgs& args, const CUtensorMap& act,
-                         const CUtensorMap& lora_act, int num_sms, cudaStream_t stream) {
+                         const CUtensorMap& lora_act, const CUtensorMap& codes_map, int num_sms,
+                         cudaStream_t stream) {
   if (dir == FusedDir::kFwd) {
     // the decode-shaped forward (16 tokens or fewer) is k_gemv's
-    if (token_tile == 256) return launch_fused_t<0, 256>(args, act, lora_act, num_sms, stream);
+    if (token_tile == 256) return launch_fused_t<0, 256>(args, act, lora_act, codes_map, num_sms, stream);
   } else {
-    if (token_tile == 256) return launch_fused_t<1, 256>(args, act, lora_act, num_sms, stream);
-    if (token_tile == 16) return launch_fused_t<1, 16>(args, act, lora_act, num_sms, stream);
+    if (token_tile == 256) return launch_fused_t<1, 256>(args, act, lora_act, codes_map, num_sms, stream);
+    if (token_tile == 16) return launch_fused_t<1, 16>(args, act, lora_act, codes_map, num_sms, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -46,8 +46,11 @@ struct FusedArgs {
 
 // Token tile of the fused kernel: 256 for prefill-shaped calls; the backward
 // also takes 16 for decode-shaped calls (M <= 16).
+// codes_map: the packed codes as uint8 [nw, kw/2], no swizzle, box {32, 128}
+// (forward) or {64, 64} (backward).
 cudaError_t launch_fused(FusedDir dir, int token_tile, const FusedArgs& args, const CUtensorMap& act,
-                         const CUtensorMap& lora_act, int num_sms, cudaStream_t stream);
+                         const CUtensorMap& lora_act, const CUtensorMap& codes_map, int num_sms,
+                         cudaStream_t stream);
 // out[i * ld_out + j] = bf16(scale * in[i * ld_in + j]) for j < cols_in, 0 for
 // cols_in <= j < cols_out (i < rows): the decode backward's split-K dX.  The
 // grid is at most 8 CTAs of 256 threads per SM (num_sms: the device's SM count).
