@@ -80,26 +80,6 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
                "r"(v.w) : "memory");
 }
 
-// L2 policy for the packed codes: every token tile of a launch re-reads the
-// whole weight, so it is kept in L2 ahead of the streamed output.
-__device__ __forceinline__ uint64_t l2_evict_last_policy() {
-  uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
-__device__ __forceinline__ uint4 ldg_nc_v4(const void* p, uint64_t pol) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p), "l"(pol));
-  return v;
-}
-// 32 bytes in one request (sm_100 256-bit load); p must be 32-byte aligned.
-__device__ __forceinline__ void ldg_nc_v8(const void* p, uint64_t pol, uint4& lo, uint4& hi) {
-  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8], %9;"
-               : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
-               : "l"(p), "l"(pol));
-}
-
 __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
@@ -115,11 +95,10 @@ struct DqLoad {
   bool valid;
 };
 
-// A block's 32 code bytes start at a multiple of 32 bytes of the code array,
-// so with a 32-byte aligned array they take one 256-bit load (one L2 request
-// per row instead of two; measured +3% on the fused kernel), else two.
+// The task's block constant and c2 (its 32 code bytes arrive by TMA: with a
+// load per thread, one L2 request per row, the kernel ran 4-5% slower).
 template <int kDir>
-__device__ __forceinline__ DqLoad dq_load(const FusedArgs& a, int m0, int kstep, int t, uint64_t pol) {
+__device__ __forceinline__ DqLoad dq_load(const FusedArgs& a, int m0, int kstep, int t) {
   DqLoad d;
   int64_t n, kcol;
   if (kDir == 0) {              // forward: task = W row m0 + t, block kstep
@@ -132,7 +111,6 @@ __device__ __forceinline__ DqLoad dq_load(const FusedArgs& a, int m0, int kstep,
   d.valid = (n < a.nw) && (kcol < a.kw);
   if (d.valid) {
     const int64_t e = n * a.kw + kcol;                 // first weight of the block
-    (void)pol;
     const int64_t blk = e >> 6;
     if (a.absf) {                 // no double quantization: the constant itself
       d.q = 0;
@@ -262,7 +240,6 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
     const int t = threadIdx.x & 127;
     const bool plain = a.absf != nullptr;
     const float mu = plain ? 0.0f : __ldg(a.mean);
-    const uint64_t codes_pol = l2_evict_last_policy();
     // The group's code tiles come by TMA into two slots, one task ahead.  A
     // slot is refilled only after this thread's wait on `empty` for the current
     // task, which implies every thread of the group has finished the task
@@ -283,14 +260,14 @@ k_fused(const FusedArgs a, const __grid_constant__ CUtensorMap act,
       int j = static_cast<int>((static_cast<uint32_t>(group) - gctr) & (kDequantGroups - 1));
       DqLoad next;
       if (j < w.kmain) {
-        next = dq_load<kDir>(a, m0, w.kbeg + j, t, codes_pol);
+        next = dq_load<kDir>(a, m0, w.kbeg + j, t);
         if (t == 0) issue_codes(ci, m0, w.kbeg + j);
       }
       for (; j < w.nk; j += kDequantGroups) {
         const uint32_t it = gctr + j;
         const uint32_t stage = it % kStages, phase = (it / kStages) & 1u;
         DqLoad cur = next;
-        if (j + kDequantGroups < w.kmain) next = dq_load<kDir>(a, m0, w.kbeg + j + kDequantGroups, t, codes_pol);
+        if (j + kDequantGroups < w.kmain) next = dq_load<kDir>(a, m0, w.kbeg + j + kDequantGroups, t);
         if (!mbar_wait(&empty[stage], phase ^ 1u, a.err)) { alive = false; break; }
         if (t == 0 && j + kDequantGroups < w.kmain) issue_codes(ci + 1, m0, w.kbeg + j + kDequantGroups);
         const uint32_t sA = smem0 + stage * kStageBytes;

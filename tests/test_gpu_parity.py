@@ -312,9 +312,9 @@ def test_results_are_bit_reproducible(qb, n, k, m):
 
 @pytest.mark.parametrize("m", [64, 8])
 def test_codes_at_a_16_byte_offset_give_identical_results(qb, m):
-    """The fused kernel loads a block's 32 code bytes in one 256-bit load when
-    the code array is 32-byte aligned and in two 128-bit loads otherwise; both
-    paths give the same bits."""
+    """The fused kernel takes its code tiles by TMA straight from the code
+    array; an array at a 16-byte offset (the least alignment the ABI accepts)
+    gives the same bits as an aligned one, forward and backward."""
     import dataclasses
     n, k, r = 392, 640, 64
     W = workloads.weight((n, k), proj=3).cuda()
